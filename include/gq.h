@@ -1,0 +1,232 @@
+/*
+ * gq.h -- libgq: per-row / per-tensor int6 and int8 weight quantization on
+ * NVIDIA B200 (sm_100a).  C ABI: plain pointers and sizes only.
+ *
+ * What the library computes follows the parameter-golf pages:
+ *  - "SubSixteen v2: Int6 QAT + MLP 3x + SWA + Sliding Window" (PR #69),
+ *    "Training Techniques / Quantization" (STE QAT, bits 6) and "Other"
+ *    (straight-through estimator fake quantization in the forward pass,
+ *    quant_range [-31, 31]);
+ *  - "Swiglu gating_ QAT_Residual Attention Scalin _EMA- Sliding window_
+ *    Optimizations for 10min/16MB Track" (PR #2159), "Key Explored
+ *    Modifications" 1 (STE fake quantization), 13 (int8 export), 14 (per-row
+ *    / per-tensor quantization), 15 (percentile clipping for the export),
+ *    16 (small-tensor FP16 passthrough), and "Final Observed Results" (int8
+ *    export validation: dequantize what was exported);
+ *  - "Record: Unified Attention + FA3 + Legal TTT" (PR #1202),
+ *    "Quantization" (int8 embeddings, int6 STE QAT on all weights);
+ *  - "Add non-record submission: 12L 24min Vocab1792 ... Int6AWQ MixedBits"
+ *    (PR #1495), "Mixed-bit quantization details" (int6 by default, tensors
+ *    named in QUANT_INT8_NAME_PATTERNS promoted to int8; default list
+ *    tok_emb.weight, lm_head.weight).
+ *
+ * The pages give no formulas.  The definitions used throughout (they are the
+ * plainest readings of the pages):
+ *   group    one row (GQ_PER_ROW) or the whole tensor (GQ_PER_TENSOR),
+ *            n elements;
+ *   k        min(n, max(1, ceil(p * n))), p * n one IEEE double multiply,
+ *            p in (0, 1];
+ *   clip c   the k-th smallest |w| of the group (1-indexed order statistic;
+ *            p = 1 gives max |w|);
+ *   qmax     31 for int6, 127 for int8 (symmetric; -32 / -128 never occur);
+ *   scale    s32 = c / qmax (binary32 division).  Export mode stores
+ *            h = binary16(s32) (round to nearest even) and uses s = (float)h to
+ *            quantize and to dequantize; training mode uses s = s32;
+ *   code     q = clamp(round_half_even(clip(w, -c, c) / s), -qmax, qmax),
+ *            binary32 division; s = 0 gives q = 0;
+ *   w_hat    (float)q * s (binary32 multiply; q = 0 gives +0.0); bf16 tensors
+ *            are widened exactly, computed in binary32, and w_hat is rounded
+ *            to bf16 (nearest even);
+ *   packing  int6: 4 codes in 3 bytes, 6-bit two's complement fields, first
+ *            code in the least significant bits of a little-endian 24-bit
+ *            group, last group of a row zero-padded, row stride
+ *            3 * ceil(cols / 4) bytes; int8: the code bytes.
+ * Every output is bit-exact to that definition.
+ *
+ * Conventions for every entry point:
+ *  - All pointers named d_* or held in gq_tensor are DEVICE pointers owned by
+ *    the caller; the gq_tensor array itself is HOST memory, read during the
+ *    call only.  The library allocates no memory and keeps no state beyond a
+ *    cached per-device property query.
+ *  - Calls are asynchronous on `stream` and never synchronize.
+ *  - Argument errors are returned before anything is launched (nothing is
+ *    written).  A failed launch returns GQ_ERR_CUDA.
+ *  - Conditions found on the device (non-finite input, a binary16 scale
+ *    overflow) are OR-ed into d_status[i] (one int32 per descriptor, nullable)
+ *    as GQ_STATUS_* bits; the call clears d_status[0..n) on the stream first.
+ *    The outputs of a descriptor whose status is non-zero are unspecified.
+ *  - Outputs are dense row-major [rows, cols] (packed: [rows, packed row
+ *    bytes]); the input may be strided (ld >= cols elements).
+ *  - A tensor with rows == 0 or cols == 0 is a no-op; its pointers may be NULL.
+ *  - No call synchronizes, spins, traps or asserts on the device.
+ */
+#ifndef GQ_H
+#define GQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Exported entry points (the library is built with hidden default visibility). */
+#if defined(__GNUC__)
+#define GQ_API __attribute__((visibility("default")))
+#else
+#define GQ_API
+#endif
+
+/* Same type as the CUDA runtime's cudaStream_t (NULL = legacy default stream). */
+typedef struct CUstream_st* cudaStream_t;
+
+typedef enum gq_status {
+    GQ_OK = 0,
+    GQ_ERR_INVALID_ARG = 1,   /* null required pointer, bad enum, p, ld, n */
+    GQ_ERR_UNSUPPORTED = 2,   /* valid request this build does not serve */
+    GQ_ERR_MISALIGNED = 3,    /* a pointer violates its stated alignment */
+    GQ_ERR_WORKSPACE = 4,     /* workspace missing or smaller than required */
+    GQ_ERR_RANGE = 5,         /* reserved (device-side: GQ_STATUS_RANGE) */
+    GQ_ERR_NONFINITE = 6,     /* reserved (device-side: GQ_STATUS_NONFINITE) */
+    GQ_ERR_CUDA = 7,          /* a CUDA runtime call or launch failed */
+    GQ_ERR_TIMEOUT = 8        /* reserved: no call waits on the device */
+} gq_status;
+
+typedef enum gq_dtype { GQ_F32 = 0, GQ_BF16 = 1 } gq_dtype;
+typedef enum gq_gran { GQ_PER_ROW = 0, GQ_PER_TENSOR = 1 } gq_gran;
+typedef enum gq_scale_mode {
+    GQ_SCALE_F32 = 0,         /* training: s = c / qmax in binary32 */
+    GQ_SCALE_F16 = 1          /* export: s = (float)binary16(c / qmax) */
+} gq_scale_mode;
+
+/* Bits OR-ed into d_status[i]. */
+#define GQ_STATUS_NONFINITE 0x1  /* a NaN or +-inf in the tensor */
+#define GQ_STATUS_RANGE     0x2  /* binary16(c / qmax) overflowed to inf */
+
+/* Kinds returned by gq_plan_kind. */
+#define GQ_KIND_RAW  0  /* not floating point: stored as is */
+#define GQ_KIND_FP16 1  /* small tensor: binary16 passthrough */
+#define GQ_KIND_INT8 2  /* name matched a promotion pattern: int8 per row */
+#define GQ_KIND_INT6 3  /* default: int6 per row */
+
+/*
+ * One tensor of a batch.  w and every output are device pointers.
+ *   w          input, row-major [rows, ld] of dtype, first cols used
+ *   dtype      GQ_F32 or GQ_BF16
+ *   qbits      6 or 8; 16 means binary16 passthrough (gq_export_pack only)
+ *   gran       GQ_PER_ROW or GQ_PER_TENSOR
+ *   p          percentile in (0, 1]; 1 = absolute maximum
+ *   dq         nullable: w_hat [rows, cols], same dtype as w
+ *   codes      nullable: int8 codes [rows, cols]
+ *   packed     nullable: [rows, gq_packed_row_bytes(cols, qbits)] bytes;
+ *              for qbits 16 it receives binary16 [rows, cols]
+ *   scale_f16  nullable: binary16 scales [groups] (export mode only)
+ *   scale_f32  nullable: the binary32 scale used, [groups]
+ *   clip       nullable: the clip value c, [groups]
+ * groups = rows for GQ_PER_ROW, 1 for GQ_PER_TENSOR.
+ * Alignment: element pointers must be aligned to their element size; 16-byte
+ * aligned rows take the vectorised path.
+ */
+typedef struct gq_tensor {
+    const void* w;
+    int32_t dtype;
+    int32_t qbits;
+    int32_t gran;
+    int32_t reserved;         /* must be 0 */
+    int64_t rows;
+    int64_t cols;
+    int64_t ld;
+    double p;
+    void* dq;
+    int8_t* codes;
+    uint8_t* packed;
+    uint16_t* scale_f16;
+    float* scale_f32;
+    float* clip;
+} gq_tensor;
+
+/*
+ * Percentile clip selection alone: writes t[i].clip (required) and, when
+ * given, nothing else.  Per-tensor descriptors need workspace
+ * (gq_workspace_size).  Source: percentile clipping, "Swiglu gating_ QAT_..."
+ * page, Key Explored Modifications 15; per-row / per-tensor, item 14.
+ */
+GQ_API gq_status gq_row_clip_select(const gq_tensor* t, int n, void* d_ws,
+                             size_t ws_bytes, int32_t* d_status,
+                             cudaStream_t stream);
+
+/*
+ * STE fake-quant forward: clip, scale, round, clamp, dequantize.  t[i].dq is
+ * required; codes, clip, scale_f32 (and scale_f16 in GQ_SCALE_F16 mode) are
+ * optional extra outputs; packed must be NULL; qbits 6 or 8.  Source: "STE
+ * QAT bits 6" and quant_range [-31, 31] ("SubSixteen v2", sections
+ * "Quantization" and "Other"); "STE QAT bits 6 scope all" (PR #1202).
+ */
+GQ_API gq_status gq_fakequant_fwd(const gq_tensor* t, int n, gq_scale_mode mode,
+                           void* d_ws, size_t ws_bytes, int32_t* d_status,
+                           cudaStream_t stream);
+
+/*
+ * Straight-through backward: g_w = g_out (accumulate = 0, bitwise copy) or
+ * g_w = g_w + g_out (accumulate = 1, one binary32 add, rounded back to bf16
+ * for GQ_BF16).  numel elements, dense.  Source: the straight-through
+ * estimator of "SubSixteen v2", section "Other": the fake-quant step is
+ * treated as the identity in the backward pass.
+ */
+GQ_API gq_status gq_ste_bwd(const void* d_g_out, void* d_g_w, gq_dtype dtype,
+                     int64_t numel, int accumulate, cudaStream_t stream);
+
+/*
+ * Export: export-mode (binary16 scale) quantization with packed output.
+ * qbits 6/8: packed and scale_f16 are required; dq, codes, clip, scale_f32
+ * optional.  qbits 16: binary16 passthrough of w into packed (read as
+ * uint16 [rows, cols]); no other output.  Source: int8 + zlib export,
+ * per-row / per-tensor, percentile clipping and FP16 passthrough ("Swiglu
+ * gating_ QAT_..." page, items 13-16); int6 export ("SubSixteen v2"); mixed
+ * int6 / int8 export ("... Int6AWQ MixedBits", Mixed-bit quantization
+ * details).
+ */
+GQ_API gq_status gq_export_pack(const gq_tensor* t, int n, void* d_ws,
+                         size_t ws_bytes, int32_t* d_status,
+                         cudaStream_t stream);
+
+/*
+ * Dequant on load: out[r, c] = (float)q[r, c] * (float)scale_f16[r] (or
+ * scale_f16[0] for GQ_PER_TENSOR), codes read from packed rows of
+ * gq_packed_row_bytes(cols, qbits) bytes; bitwise equal to the w_hat of the
+ * export call that produced them.  Source: "Successful int8 + zlib export
+ * validation" ("Swiglu gating_ QAT_..." page, Final Observed Results).
+ */
+GQ_API gq_status gq_dequant(const uint8_t* d_packed, const uint16_t* d_scale_f16,
+                     int qbits, gq_gran gran, int64_t rows, int64_t cols,
+                     void* d_out, gq_dtype out_dtype, cudaStream_t stream);
+
+/* Device workspace bytes a batch needs (0 when it has no per-tensor group). */
+GQ_API size_t gq_workspace_size(const gq_tensor* t, int n);
+
+/* Bytes of one packed row: 3*ceil(cols/4) (qbits 6), cols (8), 2*cols (16);
+ * -1 for another qbits or cols < 0. */
+GQ_API int64_t gq_packed_row_bytes(int64_t cols, int qbits);
+
+/* k = min(n, max(1, ceil(p * n))) in IEEE double; -1 if n < 1 or p not in (0, 1]. */
+GQ_API int64_t gq_k_from_p(int64_t n, double p);
+
+/*
+ * Export plan for one named tensor (host only): GQ_KIND_RAW if not floating
+ * point, GQ_KIND_FP16 if numel < small_numel, GQ_KIND_INT8 if any
+ * comma-separated pattern (NULL: "tok_emb.weight,lm_head.weight") is a
+ * substring of name, else GQ_KIND_INT6.  -1 on a bad argument.  Source:
+ * "... Int6AWQ MixedBits" (Mixed-bit quantization details) and FP16
+ * passthrough ("Swiglu gating_ QAT_..." item 16).
+ */
+GQ_API int gq_plan_kind(const char* name, const int64_t* shape, int ndim,
+                 int is_float, const char* patterns, int64_t small_numel);
+
+/* Static text for a status code. */
+GQ_API const char* gq_status_string(gq_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQ_H */

@@ -1,0 +1,408 @@
+// gq_api.cu -- the libgq C ABI (include/gq.h): argument checks, launch
+// planning and kernel launches.  Host code only; kernels are in
+// gq_kernels.cuh.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "gq.h"
+#include "gq_kernels.cuh"
+
+namespace {
+
+using namespace gq;
+
+constexpr size_t kWsSlot = 8448;      // 2048 x u32 histogram + 16 x u32 state, 256-aligned
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sm_count[kMaxDevices];
+
+int sm_count() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+    int v = g_sm_count[dev].load(std::memory_order_relaxed);
+    if (v <= 0) {
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+            v = 148;
+        g_sm_count[dev].store(v, std::memory_order_relaxed);
+    }
+    return v;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int64_t k_from_p(int64_t n, double p) {
+    double prod = p * (double)n;
+    double up = std::ceil(prod);
+    int64_t k = (int64_t)up;
+    if (k < 1) k = 1;
+    if (k > n) k = n;
+    return k;
+}
+
+int64_t packed_row_bytes(int64_t cols, int qbits) {
+    if (cols < 0) return -1;
+    if (qbits == 6) return 3 * ((cols + 3) / 4);
+    if (qbits == 8) return cols;
+    if (qbits == 16) return 2 * cols;
+    return -1;
+}
+
+enum class Op { Select, FakeQuant, Export };
+
+// Validate one descriptor for an operation.  Returns GQ_OK or an error.
+gq_status check_tensor(const gq_tensor& t, Op op, bool f16_mode) {
+    if (t.reserved != 0) return GQ_ERR_INVALID_ARG;
+    if (t.dtype != GQ_F32 && t.dtype != GQ_BF16) return GQ_ERR_INVALID_ARG;
+    if (t.gran != GQ_PER_ROW && t.gran != GQ_PER_TENSOR) return GQ_ERR_INVALID_ARG;
+    const bool pass16 = t.qbits == 16;
+    if (!(t.qbits == 6 || t.qbits == 8 || (pass16 && op == Op::Export))) return GQ_ERR_INVALID_ARG;
+    if (t.rows < 0 || t.cols < 0 || t.ld < t.cols) return GQ_ERR_INVALID_ARG;
+    if (t.cols > (int64_t)INT32_MAX) return GQ_ERR_UNSUPPORTED;
+    if (!pass16 && !(t.p > 0.0 && t.p <= 1.0)) return GQ_ERR_INVALID_ARG;
+    const int64_t esz = t.dtype == GQ_F32 ? 4 : 2;
+    if (t.rows > 0 && t.ld > 0 && t.rows > INT64_MAX / 16 / t.ld) return GQ_ERR_INVALID_ARG;
+    if (t.rows > 0 && t.cols > 0 && t.rows > INT64_MAX / 16 / t.cols) return GQ_ERR_INVALID_ARG;
+    if (t.rows == 0 || t.cols == 0) return GQ_OK;   // empty: nothing read or written
+    if (!t.w) return GQ_ERR_INVALID_ARG;
+    if (!aligned(t.w, esz)) return GQ_ERR_MISALIGNED;
+    if (t.dq && !aligned(t.dq, esz)) return GQ_ERR_MISALIGNED;
+    if (t.scale_f16 && !aligned(t.scale_f16, 2)) return GQ_ERR_MISALIGNED;
+    if (t.scale_f32 && !aligned(t.scale_f32, 4)) return GQ_ERR_MISALIGNED;
+    if (t.clip && !aligned(t.clip, 4)) return GQ_ERR_MISALIGNED;
+    switch (op) {
+        case Op::Select:
+            if (!t.clip) return GQ_ERR_INVALID_ARG;
+            if (t.dq || t.codes || t.packed || t.scale_f16 || t.scale_f32) return GQ_ERR_INVALID_ARG;
+            break;
+        case Op::FakeQuant:
+            if (!t.dq || t.packed) return GQ_ERR_INVALID_ARG;
+            if (t.scale_f16 && !f16_mode) return GQ_ERR_INVALID_ARG;
+            break;
+        case Op::Export:
+            if (pass16) {
+                if (!t.packed || t.dq || t.codes || t.scale_f16 || t.scale_f32 || t.clip)
+                    return GQ_ERR_INVALID_ARG;
+                if (!aligned(t.packed, 2)) return GQ_ERR_MISALIGNED;
+            } else if (!t.packed || !t.scale_f16) {
+                return GQ_ERR_INVALID_ARG;
+            }
+            break;
+    }
+    return GQ_OK;
+}
+
+bool needs_workspace(const gq_tensor& t) {
+    return t.qbits != 16 && t.gran == GQ_PER_TENSOR && t.rows > 0 && t.cols > 0;
+}
+
+size_t workspace_size(const gq_tensor* t, int n) {
+    size_t slots = 0;
+    for (int i = 0; i < n; ++i)
+        if (needs_workspace(t[i])) ++slots;
+    return slots * kWsSlot;
+}
+
+gq_status launch_status() {
+    return cudaGetLastError() == cudaSuccess ? GQ_OK : GQ_ERR_CUDA;
+}
+
+// Per-tensor radix select for every per-tensor descriptor (three passes).
+gq_status run_per_tensor_select(const std::vector<SelDesc>& sel, cudaStream_t stream) {
+    for (size_t base = 0; base < sel.size(); base += kMaxDesc) {
+        SelParams P;
+        std::memset(&P, 0, sizeof(P));
+        const int nd = (int)std::min<size_t>(kMaxDesc, sel.size() - base);
+        P.ndesc = nd;
+        int64_t acc = 0;
+        for (int i = 0; i < nd; ++i) {
+            P.start[i] = acc;
+            P.d[i] = sel[base + i];
+            acc += P.d[i].items;
+        }
+        P.start[nd] = acc;
+        if (acc == 0) continue;
+        if (acc > INT32_MAX) return GQ_ERR_UNSUPPORTED;
+        ptsel_kernel<0><<<(unsigned)acc, kBlockThreads, 0, stream>>>(P);
+        ptsel_kernel<1><<<(unsigned)acc, kBlockThreads, 0, stream>>>(P);
+        ptsel_kernel<2><<<(unsigned)acc, kBlockThreads, 0, stream>>>(P);
+        if (launch_status() != GQ_OK) return GQ_ERR_CUDA;
+    }
+    return GQ_OK;
+}
+
+template <int TW>
+gq_status run_rows(const std::vector<RowDesc>& rows, cudaStream_t stream) {
+    constexpr int kTeams = kBlockWarps / TW;
+    const int64_t max_blocks = (int64_t)sm_count() * (2048 / kBlockThreads);
+    for (size_t base = 0; base < rows.size(); base += kMaxDesc) {
+        RowParams P;
+        std::memset(&P, 0, sizeof(P));
+        const int nd = (int)std::min<size_t>(kMaxDesc, rows.size() - base);
+        P.ndesc = nd;
+        int64_t acc = 0;
+        for (int i = 0; i < nd; ++i) {
+            P.start[i] = acc;
+            P.d[i] = rows[base + i];
+            acc += P.d[i].items;
+        }
+        P.start[nd] = acc;
+        if (acc == 0) continue;
+        const int64_t blocks = std::min<int64_t>(max_blocks, (acc + kTeams - 1) / kTeams);
+        rowquant_kernel<TW><<<(unsigned)blocks, kBlockThreads, 0, stream>>>(P);
+        if (launch_status() != GQ_OK) return GQ_ERR_CUDA;
+    }
+    return GQ_OK;
+}
+
+gq_status run_passthrough(const std::vector<PassDesc>& pd, cudaStream_t stream) {
+    for (size_t base = 0; base < pd.size(); base += kMaxDesc) {
+        PassParams P;
+        std::memset(&P, 0, sizeof(P));
+        const int nd = (int)std::min<size_t>(kMaxDesc, pd.size() - base);
+        P.ndesc = nd;
+        int64_t acc = 0;
+        for (int i = 0; i < nd; ++i) {
+            P.start[i] = acc;
+            P.d[i] = pd[base + i];
+            acc += (P.d[i].rows * P.d[i].cols + kPassChunk - 1) / kPassChunk;
+        }
+        P.start[nd] = acc;
+        if (acc == 0) continue;
+        const int64_t blocks = std::min<int64_t>((int64_t)sm_count() * 8, acc);
+        passthrough_kernel<<<(unsigned)blocks, kBlockThreads, 0, stream>>>(P);
+        if (launch_status() != GQ_OK) return GQ_ERR_CUDA;
+    }
+    return GQ_OK;
+}
+
+// The shared driver of gq_row_clip_select, gq_fakequant_fwd and gq_export_pack.
+gq_status quantize_batch(const gq_tensor* t, int n, Op op, bool f16_mode, void* ws,
+                         size_t ws_bytes, int32_t* d_status, cudaStream_t stream) {
+    if (n < 0 || (n > 0 && !t)) return GQ_ERR_INVALID_ARG;
+    for (int i = 0; i < n; ++i) {
+        gq_status st = check_tensor(t[i], op, f16_mode);
+        if (st != GQ_OK) return st;
+    }
+    const size_t need = workspace_size(t, n);
+    if (need > 0) {
+        if (!ws || ws_bytes < need) return GQ_ERR_WORKSPACE;
+        if (!aligned(ws, 256)) return GQ_ERR_MISALIGNED;
+    }
+    if (d_status && !aligned(d_status, 4)) return GQ_ERR_MISALIGNED;
+    if (n == 0) return GQ_OK;
+
+    if (d_status && cudaMemsetAsync(d_status, 0, sizeof(int32_t) * (size_t)n, stream) != cudaSuccess)
+        return GQ_ERR_CUDA;
+    if (need > 0 && cudaMemsetAsync(ws, 0, need, stream) != cudaSuccess) return GQ_ERR_CUDA;
+
+    std::vector<SelDesc> sel;
+    std::vector<RowDesc> rows_w, rows_c;   // warp teams / block teams
+    std::vector<PassDesc> pass;
+    size_t slot = 0;
+    for (int i = 0; i < n; ++i) {
+        const gq_tensor& T = t[i];
+        if (T.rows == 0 || T.cols == 0) continue;
+        const int esz = T.dtype == GQ_F32 ? 4 : 2;
+        int32_t* status = d_status ? d_status + i : nullptr;
+        if (T.qbits == 16) {
+            PassDesc P{};
+            P.w = T.w;
+            P.out = reinterpret_cast<uint16_t*>(T.packed);
+            P.rows = T.rows;
+            P.cols = T.cols;
+            P.ld = T.ld;
+            P.dtype = T.dtype;
+            pass.push_back(P);
+            continue;
+        }
+        RowDesc D{};
+        D.w = T.w;
+        D.dq = T.dq;
+        D.codes = T.codes;
+        D.packed = T.packed;
+        D.sf16 = (op == Op::FakeQuant && !f16_mode) ? nullptr : T.scale_f16;
+        D.sf32 = T.scale_f32;
+        D.clip_out = T.clip;
+        D.status = status;
+        D.rows = T.rows;
+        D.cols = T.cols;
+        D.ld = T.ld;
+        D.prb = packed_row_bytes(T.cols, T.qbits);
+        D.qmax = T.qbits == 6 ? 31 : 127;
+        D.dtype = T.dtype;
+        D.qbits = T.qbits;
+        D.export_mode = (op == Op::Export || f16_mode) ? 1 : 0;
+        const bool elem = T.dq || T.codes || T.packed;
+        int32_t flags = elem ? kElemOut : 0;
+        const size_t vin = T.dtype == GQ_F32 ? 16 : 8;
+        if (aligned(T.w, vin) && ((T.ld * esz) % (int64_t)vin) == 0) flags |= kVecIn;
+        if (T.dq && aligned(T.dq, vin) && ((T.cols * esz) % (int64_t)vin) == 0) flags |= kVecDq;
+        if (T.codes && aligned(T.codes, 4) && (T.cols % 4) == 0) flags |= kVecCodes;
+        if (T.packed && aligned(T.packed, 4) && (D.prb % 4) == 0) flags |= kVecPacked;
+        if (T.gran == GQ_PER_TENSOR) {
+            flags |= kPerTensor;
+            const int64_t numel = T.rows * T.cols;
+            uint8_t* base = static_cast<uint8_t*>(ws) + slot * kWsSlot;
+            ++slot;
+            SelDesc S{};
+            S.w = T.w;
+            S.hist = reinterpret_cast<uint32_t*>(base);
+            S.state = reinterpret_cast<uint32_t*>(base + kSelBins * sizeof(uint32_t));
+            S.status = status;
+            S.rows = T.rows;
+            S.cols = T.cols;
+            S.ld = T.ld;
+            S.rows_per_item = std::max<int64_t>(1, 65536 / T.cols);
+            S.items = (T.rows + S.rows_per_item - 1) / S.rows_per_item;
+            S.m = numel - k_from_p(numel, T.p) + 1;
+            S.dtype = T.dtype;
+            sel.push_back(S);
+            D.clip_in = S.state + 3;
+            D.m = 0;
+            D.items = elem ? T.rows : 1;
+        } else {
+            D.m = (int32_t)(T.cols - k_from_p(T.cols, T.p) + 1);
+            D.items = T.rows;
+        }
+        D.flags = flags;
+        if (T.cols <= 2048)
+            rows_w.push_back(D);
+        else
+            rows_c.push_back(D);
+    }
+
+    gq_status st = run_per_tensor_select(sel, stream);
+    if (st != GQ_OK) return st;
+    st = run_rows<1>(rows_w, stream);
+    if (st != GQ_OK) return st;
+    st = run_rows<kBlockWarps>(rows_c, stream);
+    if (st != GQ_OK) return st;
+    return run_passthrough(pass, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+gq_status gq_row_clip_select(const gq_tensor* t, int n, void* d_ws, size_t ws_bytes,
+                             int32_t* d_status, cudaStream_t stream) {
+    return quantize_batch(t, n, Op::Select, false, d_ws, ws_bytes, d_status, stream);
+}
+
+gq_status gq_fakequant_fwd(const gq_tensor* t, int n, gq_scale_mode mode, void* d_ws,
+                           size_t ws_bytes, int32_t* d_status, cudaStream_t stream) {
+    if (mode != GQ_SCALE_F32 && mode != GQ_SCALE_F16) return GQ_ERR_INVALID_ARG;
+    return quantize_batch(t, n, Op::FakeQuant, mode == GQ_SCALE_F16, d_ws, ws_bytes, d_status,
+                          stream);
+}
+
+gq_status gq_export_pack(const gq_tensor* t, int n, void* d_ws, size_t ws_bytes,
+                         int32_t* d_status, cudaStream_t stream) {
+    return quantize_batch(t, n, Op::Export, true, d_ws, ws_bytes, d_status, stream);
+}
+
+gq_status gq_ste_bwd(const void* d_g_out, void* d_g_w, gq_dtype dtype, int64_t numel,
+                     int accumulate, cudaStream_t stream) {
+    if (dtype != GQ_F32 && dtype != GQ_BF16) return GQ_ERR_INVALID_ARG;
+    if (numel < 0 || (accumulate != 0 && accumulate != 1)) return GQ_ERR_INVALID_ARG;
+    if (numel == 0) return GQ_OK;
+    if (!d_g_out || !d_g_w) return GQ_ERR_INVALID_ARG;
+    const size_t esz = dtype == GQ_F32 ? 4 : 2;
+    if (!aligned(d_g_out, esz) || !aligned(d_g_w, esz)) return GQ_ERR_MISALIGNED;
+    if ((uint64_t)numel > (uint64_t)INT64_MAX / 16) return GQ_ERR_INVALID_ARG;
+    const int vec = aligned(d_g_out, 16) && aligned(d_g_w, 16);
+    const int64_t per = dtype == GQ_F32 ? 4 : 8;
+    const int64_t units = vec ? (numel + per - 1) / per : numel;
+    const int64_t blocks = std::min<int64_t>((int64_t)sm_count() * 8,
+                                             std::max<int64_t>(1, (units + kBlockThreads - 1) / kBlockThreads));
+    ste_kernel<<<(unsigned)blocks, kBlockThreads, 0, stream>>>(d_g_out, d_g_w, dtype, numel,
+                                                                accumulate, vec);
+    return launch_status();
+}
+
+gq_status gq_dequant(const uint8_t* d_packed, const uint16_t* d_scale_f16, int qbits,
+                     gq_gran gran, int64_t rows, int64_t cols, void* d_out,
+                     gq_dtype out_dtype, cudaStream_t stream) {
+    if (qbits != 6 && qbits != 8) return GQ_ERR_INVALID_ARG;
+    if (gran != GQ_PER_ROW && gran != GQ_PER_TENSOR) return GQ_ERR_INVALID_ARG;
+    if (out_dtype != GQ_F32 && out_dtype != GQ_BF16) return GQ_ERR_INVALID_ARG;
+    if (rows < 0 || cols < 0) return GQ_ERR_INVALID_ARG;
+    if (rows == 0 || cols == 0) return GQ_OK;
+    if (!d_packed || !d_scale_f16 || !d_out) return GQ_ERR_INVALID_ARG;
+    if (rows > INT64_MAX / 16 / cols) return GQ_ERR_INVALID_ARG;
+    const size_t esz = out_dtype == GQ_F32 ? 4 : 2;
+    if (!aligned(d_scale_f16, 2) || !aligned(d_out, esz)) return GQ_ERR_MISALIGNED;
+    const int64_t prb = packed_row_bytes(cols, qbits);
+    const int vec_out = out_dtype == GQ_F32 && aligned(d_out, 16) && (cols % 4) == 0;
+    const int64_t total = rows * ((cols + 3) / 4);
+    const int64_t blocks = std::min<int64_t>((int64_t)sm_count() * 8,
+                                             (total + kBlockThreads - 1) / kBlockThreads);
+    dequant_kernel<<<(unsigned)blocks, kBlockThreads, 0, stream>>>(
+        d_packed, d_scale_f16, qbits, gran == GQ_PER_TENSOR, rows, cols, prb, d_out, out_dtype,
+        vec_out);
+    return launch_status();
+}
+
+size_t gq_workspace_size(const gq_tensor* t, int n) {
+    if (!t || n <= 0) return 0;
+    return workspace_size(t, n);
+}
+
+int64_t gq_packed_row_bytes(int64_t cols, int qbits) { return packed_row_bytes(cols, qbits); }
+
+int64_t gq_k_from_p(int64_t n, double p) {
+    if (n < 1 || !(p > 0.0 && p <= 1.0)) return -1;
+    return k_from_p(n, p);
+}
+
+int gq_plan_kind(const char* name, const int64_t* shape, int ndim, int is_float,
+                 const char* patterns, int64_t small_numel) {
+    if (!name || ndim < 0 || (ndim > 0 && !shape) || small_numel < 0) return -1;
+    int64_t numel = 1;
+    for (int i = 0; i < ndim; ++i) {
+        if (shape[i] < 0) return -1;
+        numel *= shape[i];
+    }
+    if (!is_float) return GQ_KIND_RAW;
+    if (numel < small_numel) return GQ_KIND_FP16;
+    const char* pats = patterns ? patterns : "tok_emb.weight,lm_head.weight";
+    const char* p = pats;
+    while (*p) {
+        const char* comma = std::strchr(p, ',');
+        size_t len = comma ? (size_t)(comma - p) : std::strlen(p);
+        // trim spaces
+        const char* b = p;
+        const char* e = p + len;
+        while (b < e && *b == ' ') ++b;
+        while (e > b && e[-1] == ' ') --e;
+        if (e > b) {
+            std::string pat(b, (size_t)(e - b));
+            if (std::strstr(name, pat.c_str())) return GQ_KIND_INT8;
+        }
+        if (!comma) break;
+        p = comma + 1;
+    }
+    return GQ_KIND_INT6;
+}
+
+const char* gq_status_string(gq_status s) {
+    switch (s) {
+        case GQ_OK: return "ok";
+        case GQ_ERR_INVALID_ARG: return "invalid argument";
+        case GQ_ERR_UNSUPPORTED: return "unsupported";
+        case GQ_ERR_MISALIGNED: return "misaligned pointer";
+        case GQ_ERR_WORKSPACE: return "workspace missing or too small";
+        case GQ_ERR_RANGE: return "binary16 scale overflow";
+        case GQ_ERR_NONFINITE: return "non-finite input";
+        case GQ_ERR_CUDA: return "CUDA error";
+        case GQ_ERR_TIMEOUT: return "timeout";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"
