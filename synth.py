@@ -22,6 +22,7 @@ manifest order below; the bandwidth workload is drawn on the GPU from a seeded
 """
 from __future__ import annotations
 
+import functools
 import math
 from dataclasses import dataclass, field
 
@@ -52,10 +53,14 @@ def _normal(rng, n, std):
     return (rng.standard_normal(n) * std).astype(np.float32)
 
 
-def _student_t3(rng, n, std):
-    z = rng.standard_normal((4, n))
-    t = z[0] / np.sqrt((z[1] ** 2 + z[2] ** 2 + z[3] ** 2) / 3.0)
-    return (t * (std / math.sqrt(3.0))).astype(np.float32)
+def _student_t3(rng, n, std, chunk=1 << 20):
+    out = np.empty(n, np.float32)
+    for i in range(0, n, chunk):
+        m = min(chunk, n - i)
+        z = rng.standard_normal((4, m))
+        t = z[0] / np.sqrt((z[1] ** 2 + z[2] ** 2 + z[3] ** 2) / 3.0)
+        out[i:i + m] = t * (std / math.sqrt(3.0))
+    return out
 
 
 def _outlier_mix(rng, n):
@@ -157,8 +162,10 @@ def draw_single_matrix():
     return w, g
 
 
+@functools.lru_cache(maxsize=1)
 def draw_gpt9():
-    """Dict name -> fp32 array, Student-t(3) scaled to std 0.02, seed 1."""
+    """Dict name -> fp32 array, Student-t(3) scaled to std 0.02, seed 1.
+    Cached: callers must not modify the arrays."""
     rng = np.random.default_rng(1)
     out = {}
     for s in gpt9_specs():

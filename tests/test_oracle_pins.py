@@ -374,16 +374,22 @@ def test_invariants(orc):
 
 def check_pack_roundtrip_exhaustive(orc):
     """Every quadruple of codes in [-31, 31]: pack then unpack is the identity,
-    and each 3-byte group equals the little-endian 24-bit sum of 6-bit fields."""
-    v = np.arange(-31, 32, dtype=np.int8)
-    a, b, c, d = np.meshgrid(v, v, v, v, indexing="ij")
-    q = np.stack([a.ravel(), b.ravel(), c.ravel(), d.ravel()], axis=1).ravel()
-    packed = orc.pack6_row(q)
-    assert np.array_equal(orc.unpack6_row(packed, q.size), q)
-    u = (q.astype(np.int64) & 0x3F).reshape(-1, 4)
-    val = u[:, 0] | (u[:, 1] << 6) | (u[:, 2] << 12) | (u[:, 3] << 18)
-    g = packed.reshape(-1, 3).astype(np.int64)
-    assert np.array_equal(g[:, 0] | (g[:, 1] << 8) | (g[:, 2] << 16), val)
+    and each 3-byte group equals the little-endian 24-bit sum of 6-bit fields.
+    Swept in 63 chunks (first code fixed) to keep memory small."""
+    v = np.arange(-31, 32, dtype=np.int32)
+    b, c, d = np.meshgrid(v, v, v, indexing="ij")
+    rest = np.stack([b.ravel(), c.ravel(), d.ravel()], axis=1)          # 63^3 x 3
+    quad = np.empty((rest.shape[0], 4), np.int32)
+    quad[:, 1:] = rest
+    for a in range(-31, 32):
+        quad[:, 0] = a
+        q = quad.astype(np.int8).ravel()
+        packed = orc.pack6_row(q)
+        assert np.array_equal(orc.unpack6_row(packed, q.size), q)
+        u = quad & 0x3F
+        val = u[:, 0] | (u[:, 1] << 6) | (u[:, 2] << 12) | (u[:, 3] << 18)
+        g = packed.reshape(-1, 3).astype(np.int32)
+        assert np.array_equal(g[:, 0] | (g[:, 1] << 8) | (g[:, 2] << 16), val)
 
 
 def test_pack_roundtrip_exhaustive(orc):
