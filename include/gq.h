@@ -191,6 +191,34 @@ GQ_API gq_status gq_export_pack(const gq_tensor* t, int n, void* d_ws,
                          cudaStream_t stream);
 
 /*
+ * Export without any caller-provided device memory.  The paper has no
+ * counterpart: this is a convenience of this library.
+ *
+ * Same computation, arguments and outputs as gq_export_pack, but the scratch
+ * that per-tensor groups need comes from a fixed array inside the library
+ * (GQ_NOALLOC_SCRATCH_BYTES per GPU, held by every GPU that loads the library
+ * until the process exits) instead of a workspace.  It is meant for callers
+ * that cannot allocate device memory for a workspace: runtimes that own a
+ * fixed device-memory budget and hand out only the tensors themselves, code
+ * that must not trigger cudaMalloc's implicit device-wide synchronization,
+ * and plain C hosts with no allocator at hand.  It calls no cudaMalloc,
+ * cudaFree or other allocating routine.
+ *
+ *  - At most GQ_NOALLOC_MAX_PER_TENSOR per-tensor descriptors per call; a
+ *    larger batch returns GQ_ERR_WORKSPACE before anything is launched.
+ *  - The first call on a device looks up the array's device address (with
+ *    that device current) and caches it; make that first call before any
+ *    stream capture.
+ *  - All calls on a device share the one array and each call clears the part
+ *    it uses; calls whose work overlaps on the GPU (different streams, or
+ *    different host threads without ordering) race on it.
+ */
+#define GQ_NOALLOC_MAX_PER_TENSOR 64
+#define GQ_NOALLOC_SCRATCH_BYTES (64 * 8448)
+GQ_API gq_status gq_export_pack_noalloc(const gq_tensor* t, int n,
+                                        int32_t* d_status, cudaStream_t stream);
+
+/*
  * Dequant on load: out[r, c] = (float)q[r, c] * (float)scale_f16[r] (or
  * scale_f16[0] for GQ_PER_TENSOR), codes read from packed rows of
  * gq_packed_row_bytes(cols, qbits) bytes; bitwise equal to the w_hat of the

@@ -285,6 +285,29 @@ gq_status quantize_batch(const gq_tensor* t, int n, Op op, bool f16_mode, void* 
     return run_passthrough(pass, stream);
 }
 
+// Scratch of gq_export_pack_noalloc: a fixed device array that every call on
+// a device shares, for callers that cannot hand the library any device memory.
+constexpr size_t kNoAllocSlots = 64;                       // per-tensor groups per call
+constexpr size_t kNoAllocBytes = kNoAllocSlots * kWsSlot;  // 528 KiB per device
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+std::atomic<void*> g_noalloc_addr[kMaxDevices];
+
+// Device address of g_noalloc_scratch on the current device.  Host code sees
+// only a host-side stand-in for the array, so the address is looked up once
+// per device (with that device current) and cached.
+gq_status noalloc_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GQ_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return GQ_ERR_UNSUPPORTED;
+    void* p = g_noalloc_addr[dev].load(std::memory_order_acquire);
+    if (!p) {
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return GQ_ERR_CUDA;
+        g_noalloc_addr[dev].store(p, std::memory_order_release);
+    }
+    *out = p;
+    return GQ_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -304,6 +327,19 @@ gq_status gq_fakequant_fwd(const gq_tensor* t, int n, gq_scale_mode mode, void* 
 gq_status gq_export_pack(const gq_tensor* t, int n, void* d_ws, size_t ws_bytes,
                          int32_t* d_status, cudaStream_t stream) {
     return quantize_batch(t, n, Op::Export, true, d_ws, ws_bytes, d_status, stream);
+}
+
+gq_status gq_export_pack_noalloc(const gq_tensor* t, int n, int32_t* d_status,
+                                 cudaStream_t stream) {
+    if (n < 0 || (n > 0 && !t)) return GQ_ERR_INVALID_ARG;
+    const size_t need = n > 0 ? workspace_size(t, n) : 0;
+    if (need > kNoAllocBytes) return GQ_ERR_WORKSPACE;
+    void* ws = nullptr;
+    if (need > 0) {
+        gq_status st = noalloc_scratch(&ws);
+        if (st != GQ_OK) return st;
+    }
+    return quantize_batch(t, n, Op::Export, true, ws, kNoAllocBytes, d_status, stream);
 }
 
 gq_status gq_ste_bwd(const void* d_g_out, void* d_g_w, gq_dtype dtype, int64_t numel,

@@ -38,7 +38,7 @@ STATUS_NAMES = {0: "GQ_OK", 1: "GQ_ERR_INVALID_ARG", 2: "GQ_ERR_UNSUPPORTED",
                 6: "GQ_ERR_NONFINITE", 7: "GQ_ERR_CUDA", 8: "GQ_ERR_TIMEOUT"}
 
 EXPORTED = ("gq_row_clip_select", "gq_fakequant_fwd", "gq_ste_bwd", "gq_export_pack",
-            "gq_dequant", "gq_workspace_size", "gq_packed_row_bytes", "gq_k_from_p",
+            "gq_export_pack_noalloc", "gq_dequant", "gq_workspace_size", "gq_packed_row_bytes", "gq_k_from_p",
             "gq_plan_kind", "gq_status_string")
 
 
@@ -70,9 +70,11 @@ def _load() -> C.CDLL:
     L.gq_row_clip_select.argtypes = [T, i32, vp, sz, vp, vp]
     L.gq_fakequant_fwd.argtypes = [T, i32, i32, vp, sz, vp, vp]
     L.gq_export_pack.argtypes = [T, i32, vp, sz, vp, vp]
+    L.gq_export_pack_noalloc.argtypes = [T, i32, vp, vp]
     L.gq_ste_bwd.argtypes = [vp, vp, i32, i64, i32, vp]
     L.gq_dequant.argtypes = [vp, vp, i32, i32, i64, i64, vp, i32, vp]
-    for f in ("gq_row_clip_select", "gq_fakequant_fwd", "gq_export_pack", "gq_ste_bwd", "gq_dequant"):
+    for f in ("gq_row_clip_select", "gq_fakequant_fwd", "gq_export_pack", "gq_export_pack_noalloc",
+              "gq_ste_bwd", "gq_dequant"):
         getattr(L, f).restype = i32
     L.gq_workspace_size.argtypes = [T, i32]
     L.gq_workspace_size.restype = sz
@@ -125,6 +127,12 @@ def gq_fakequant_fwd(descs, mode, ws=0, ws_bytes=0, d_status=0, stream=None):
 def gq_export_pack(descs, ws=0, ws_bytes=0, d_status=0, stream=None):
     _check(LIB.gq_export_pack(_arr(descs), len(descs), ws or None, ws_bytes,
                               d_status or None, _stream(stream)), "gq_export_pack")
+
+
+def gq_export_pack_noalloc(descs, d_status=0, stream=None):
+    """gq_export_pack with the library's fixed scratch instead of a workspace."""
+    _check(LIB.gq_export_pack_noalloc(_arr(descs), len(descs), d_status or None, _stream(stream)),
+           "gq_export_pack_noalloc")
 
 
 def gq_ste_bwd(g_out_ptr, g_w_ptr, dtype, numel, accumulate, stream=None):
