@@ -12,6 +12,7 @@
 
 #include "gq.h"
 #include "gq_kernels.cuh"
+#include "gq_rowquant_tma.cuh"
 
 namespace {
 
@@ -159,6 +160,66 @@ gq_status run_rows(const std::vector<RowDesc>& rows, cudaStream_t stream) {
     return GQ_OK;
 }
 
+// Pipelined launch over the descriptors whose rows can be bulk-copied.
+constexpr int kTmaStageBytes = 64 * 1024;
+constexpr int kTmaMaxRowBytes = 96 * 1024;
+std::atomic<int> g_tma_smem_set[kMaxDevices];
+
+bool tma_eligible(const gq_tensor& T, int32_t flags) {
+    const int64_t esz = T.dtype == GQ_F32 ? 4 : 2;
+    const int64_t row_bytes = T.cols * esz;
+    return (flags & kElemOut) && aligned(T.w, 16) && ((T.ld * esz) % 16) == 0 &&
+           (row_bytes % 16) == 0 && row_bytes <= kTmaMaxRowBytes;
+}
+
+gq_status run_rows_tma(std::vector<RowDesc>& rows, cudaStream_t stream) {
+    if (rows.empty()) return GQ_OK;
+    int64_t max_row = 0;
+    for (const RowDesc& D : rows) max_row = std::max<int64_t>(max_row, D.cols * (D.dtype == kF32 ? 4 : 2));
+    const int sb = max_row <= kTmaStageBytes ? kTmaStageBytes : (int)((max_row + 15) / 16 * 16);
+    const int nstages = max_row <= kTmaStageBytes ? 3 : 2;
+    for (RowDesc& D : rows) {
+        const int64_t row_bytes = D.cols * (D.dtype == kF32 ? 4 : 2);
+        int64_t R = sb / row_bytes;
+        int G = 1;
+        while (G < kTmaConsumerWarps && kTmaConsumerWarps / G > R) G *= 2;
+        const int64_t teams = kTmaConsumerWarps / G;
+        if (R >= teams) R = R / teams * teams;
+        D.tile_rows = (int32_t)R;
+        D.team_warps = G;
+        D.items = (D.rows + R - 1) / R;
+    }
+    const size_t smem = (size_t)nstages * sb + kTmaExtraBytes;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GQ_ERR_CUDA;
+    if (dev >= 0 && dev < kMaxDevices && g_tma_smem_set[dev].load() < (int)smem) {
+        if (cudaFuncSetAttribute(rowquant_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem) != cudaSuccess)
+            return GQ_ERR_CUDA;
+        g_tma_smem_set[dev].store((int)smem);
+    }
+    for (size_t base = 0; base < rows.size(); base += kMaxDesc) {
+        TmaParams P;
+        std::memset(&P, 0, sizeof(P));
+        const int nd = (int)std::min<size_t>(kMaxDesc, rows.size() - base);
+        P.ndesc = nd;
+        P.nstages = nstages;
+        P.stage_bytes = sb;
+        int64_t acc = 0;
+        for (int i = 0; i < nd; ++i) {
+            P.start[i] = acc;
+            P.d[i] = rows[base + i];
+            acc += P.d[i].items;
+        }
+        P.start[nd] = acc;
+        if (acc == 0) continue;
+        const int64_t blocks = std::min<int64_t>(sm_count(), acc);
+        rowquant_tma_kernel<<<(unsigned)blocks, kTmaThreads, smem, stream>>>(P);
+        if (launch_status() != GQ_OK) return GQ_ERR_CUDA;
+    }
+    return GQ_OK;
+}
+
 gq_status run_passthrough(const std::vector<PassDesc>& pd, cudaStream_t stream) {
     for (size_t base = 0; base < pd.size(); base += kMaxDesc) {
         PassParams P;
@@ -202,6 +263,7 @@ gq_status quantize_batch(const gq_tensor* t, int n, Op op, bool f16_mode, void* 
 
     std::vector<SelDesc> sel;
     std::vector<RowDesc> rows_w, rows_c;   // warp teams / block teams
+    std::vector<RowDesc> rows_tma;         // pipelined through shared memory
     std::vector<PassDesc> pass;
     size_t slot = 0;
     for (int i = 0; i < n; ++i) {
@@ -270,13 +332,17 @@ gq_status quantize_batch(const gq_tensor* t, int n, Op op, bool f16_mode, void* 
             D.items = T.rows;
         }
         D.flags = flags;
-        if (T.cols <= 2048)
+        if (tma_eligible(T, flags))
+            rows_tma.push_back(D);
+        else if (T.cols <= 2048)
             rows_w.push_back(D);
         else
             rows_c.push_back(D);
     }
 
     gq_status st = run_per_tensor_select(sel, stream);
+    if (st != GQ_OK) return st;
+    st = run_rows_tma(rows_tma, stream);
     if (st != GQ_OK) return st;
     st = run_rows<1>(rows_w, stream);
     if (st != GQ_OK) return st;

@@ -42,6 +42,8 @@ struct RowDesc {
     int32_t qbits;
     int32_t export_mode;
     int32_t flags;             // kVec* bits
+    int32_t tile_rows;         // pipelined kernel: rows per shared-memory tile
+    int32_t team_warps;        // pipelined kernel: warps per row (power of two)
 };
 
 constexpr int32_t kVecIn = 1;       // rows of w are 16-byte (f32) / 8-byte (bf16) aligned

@@ -421,3 +421,37 @@ def test_workspace_error_on_device(gq):
     with pytest.raises(gq.GQError) as e:
         gq.gq_export_pack([d], ws=0, ws_bytes=0)
     assert e.value.status == 4
+
+
+def test_pipelined_mixed_team_sizes_one_launch(gq):
+    """One batch whose rows need every team size (1..16 warps) and both
+    dtypes: the pipelined kernel switches team shape from tile to tile."""
+    rng = np.random.default_rng(11)
+    shapes = [(70, 512), (33, 1536), (21, 4096), (5, 16384), (300, 128), (40, 528), (17, 1584)]
+    reqs, refs = [], []
+    for j, (r, c) in enumerate(shapes):
+        for dt in ("f32", "bf16"):
+            w = synth.random_matrix(rng, r, c, ("t3", "mix", "normal")[j % 3])
+            if dt == "bf16":
+                w = synth.to_bf16_bits(w).reshape(r, c)
+            p = (1.0, 0.9999, 0.99, 0.5)[(j + len(reqs)) % 4]
+            qb = 6 if (j + len(reqs)) % 3 else 8
+            reqs.append(full_request(gq, to_dev(w), qb, p))
+            refs.append((f"{r}x{c} {dt} q{qb} p{p}", oracle.quantize(w, qb, p, export=True)))
+    outs = gq.export_pack(reqs)
+    for o, (name, ref) in zip(outs, refs):
+        check_quantized(o, ref, "mixed " + name)
+
+
+def test_pipelined_strided_bf16_and_two_stage_rows(gq):
+    rng = np.random.default_rng(12)
+    full = synth.to_bf16_bits(synth.random_matrix(rng, 24, 1040, "t3")).reshape(24, 1040)
+    Wf = to_dev(full)
+    (o,) = gq.export_pack([full_request(gq, Wf[:, :1024], 6, 0.999)])   # ld 1040, rows bulk-copied one by one
+    ref = oracle.quantize(full, 6, 0.999, export=True, cols=1024)
+    check_quantized(o, ref, "strided bf16")
+    # 80 KB rows: two 80 KB stages instead of three 64 KB ones
+    w = synth.random_matrix(rng, 9, 20000, "mix")
+    run_export_and_check(gq, w, 6, 0.9999, what="two-stage 20000 cols")
+    run_train_and_check(gq, w, 8, 0.3, what="two-stage 20000 cols radix")
+    run_export_and_check(gq, w, 6, 0.999, per_tensor=True, what="two-stage per-tensor")
