@@ -161,7 +161,7 @@ gq_status run_rows(const std::vector<RowDesc>& rows, cudaStream_t stream) {
 }
 
 // Pipelined launch over the descriptors whose rows can be bulk-copied.
-constexpr int kTmaStageBytes = 64 * 1024;
+constexpr int kTmaStageBytes = 68 * 1024;
 constexpr int kTmaMaxRowBytes = 96 * 1024;
 std::atomic<int> g_tma_smem_set[kMaxDevices];
 
@@ -172,6 +172,39 @@ bool tma_eligible(const gq_tensor& T, int32_t flags) {
            (row_bytes % 16) == 0 && row_bytes <= kTmaMaxRowBytes;
 }
 
+// Output configuration of the branch-free loops, or kOutGeneric.
+int32_t tma_out_mode(const RowDesc& D) {
+    int32_t mode = 0;
+    if (D.dq) {
+        if (!(D.flags & kVecDq)) return kOutGeneric;
+        mode |= kOutDq;
+    }
+    if (D.codes) {
+        if (!(D.flags & kVecCodes)) return kOutGeneric;
+        mode |= kOutCodes;
+    }
+    if (D.packed) {
+        if (!(D.flags & kVecPacked)) return kOutGeneric;
+        if (D.qbits == 6) {
+            if (D.cols % 16 != 0) return kOutGeneric;   // partial 4-code groups
+            mode |= kOutSix;
+        }
+        mode |= kOutPacked;
+    }
+    switch (mode) {
+        case kOutDq | kOutPacked | kOutSix:
+        case kOutDq | kOutPacked:
+        case kOutDq:
+        case kOutPacked | kOutSix:
+        case kOutPacked:
+        case kOutDq | kOutCodes | kOutPacked | kOutSix:
+        case kOutDq | kOutCodes:
+            return mode;
+        default:
+            return kOutGeneric;
+    }
+}
+
 gq_status run_rows_tma(std::vector<RowDesc>& rows, cudaStream_t stream) {
     if (rows.empty()) return GQ_OK;
     int64_t max_row = 0;
@@ -180,14 +213,16 @@ gq_status run_rows_tma(std::vector<RowDesc>& rows, cudaStream_t stream) {
     const int nstages = max_row <= kTmaStageBytes ? 3 : 2;
     for (RowDesc& D : rows) {
         const int64_t row_bytes = D.cols * (D.dtype == kF32 ? 4 : 2);
-        int64_t R = sb / row_bytes;
-        int G = 1;
-        while (G < kTmaConsumerWarps && kTmaConsumerWarps / G > R) G *= 2;
-        const int64_t teams = kTmaConsumerWarps / G;
-        if (R >= teams) R = R / teams * teams;
-        D.tile_rows = (int32_t)R;
-        D.team_warps = G;
-        D.items = (D.rows + R - 1) / R;
+        const int64_t rmax = sb / row_bytes;
+        // radix selection (m > 8, per row) runs on whole warps
+        const bool whole_warps = !D.clip_in && D.m > kTopMax;
+        int lpr = 8;
+        while (lpr < kTmaConsumers && (kTmaConsumers / lpr > rmax || (whole_warps && lpr < 32))) lpr *= 2;
+        const int64_t slots = kTmaConsumers / lpr;
+        D.tile_rows = (int32_t)(rmax / slots * slots);
+        D.lanes_per_row = lpr;
+        D.out_mode = tma_out_mode(D);
+        D.items = (D.rows + D.tile_rows - 1) / D.tile_rows;
     }
     const size_t smem = (size_t)nstages * sb + kTmaExtraBytes;
     int dev = 0;
@@ -325,7 +360,7 @@ gq_status quantize_batch(const gq_tensor* t, int n, Op op, bool f16_mode, void* 
             S.dtype = T.dtype;
             sel.push_back(S);
             D.clip_in = S.state + 3;
-            D.m = 0;
+            D.m = S.m > 1 ? 2 : 1;     // clip is given; only "some |w| > c" matters
             D.items = elem ? T.rows : 1;
         } else {
             D.m = (int32_t)(T.cols - k_from_p(T.cols, T.p) + 1);

@@ -43,7 +43,9 @@ struct RowDesc {
     int32_t export_mode;
     int32_t flags;             // kVec* bits
     int32_t tile_rows;         // pipelined kernel: rows per shared-memory tile
-    int32_t team_warps;        // pipelined kernel: warps per row (power of two)
+    int32_t lanes_per_row;     // pipelined kernel: threads per row (8 .. 512)
+    int32_t out_mode;          // pipelined kernel: output configuration, -1 generic
+    int32_t pad2;
 };
 
 constexpr int32_t kVecIn = 1;       // rows of w are 16-byte (f32) / 8-byte (bf16) aligned

@@ -4,16 +4,23 @@
 // One persistent block per SM: warp 16 is the producer, warps 0..15 consume.
 // The weights are cut into tiles of whole rows (one descriptor per tile) that
 // fill a stage of a ring of shared-memory stages.  The producer's elected lane
-// issues cp.async.bulk copies global -> shared for tile i + stages - 1 while
-// the consumers work on tile i; completion is tracked by one mbarrier per
+// issues cp.async.bulk copies global -> shared for the next tiles while the
+// consumers work on the current one; completion is tracked by one mbarrier per
 // stage ("full", transaction bytes) and stages are handed back through a
 // second mbarrier ("empty", one arrival per consumer warp).  Each input byte
-// is read from HBM exactly once, with up to (stages - 1) tiles in flight per SM.
+// is read from HBM exactly once, with up to (stages - 1) tiles in flight.
 //
-// Consumers form teams of G warps (a power of two, per descriptor) that own a
-// row: the row is read from shared memory twice (selection, then quantize),
-// and every output (w_hat, int8 codes, packed int6/int8 bytes, scales) is
-// written straight from registers with coalesced vector stores.
+// A row is owned by a slot of `lpr` consumer threads (lanes per row, a power
+// of two from 8 to 512, chosen per descriptor):
+//   lpr <= 32 : 32 / lpr rows share a warp, so every per-row step (the
+//               selection butterfly, the scale, the output pointers) is one
+//               warp instruction for several rows;
+//   lpr >= 64 : G = lpr / 32 warps own a row; the first warp merges the
+//               per-warp selections and broadcasts the row's clip through
+//               shared memory (two team barriers per row).
+// The row is read from shared memory twice (selection, then quantize), and
+// every output (w_hat, int8 codes, packed int6 / int8 bytes, scales) is
+// written from registers with coalesced vector stores.
 //
 // Every wait is bounded (a few seconds of %globaltimer): on expiry the thread
 // records GQ_STATUS_TIMEOUT in the tile's status word and leaves its loop; the
@@ -26,10 +33,16 @@
 namespace gq {
 
 constexpr int kTmaConsumerWarps = 16;
-constexpr int kTmaThreads = (kTmaConsumerWarps + 1) * 32;
+constexpr int kTmaConsumers = kTmaConsumerWarps * 32;
+constexpr int kTmaThreads = kTmaConsumers + 32;
 constexpr int kTmaMaxStages = 4;
 constexpr uint32_t kStatusTimeout = 0x4u;
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;   // 4 s
+
+// Output configurations with a branch-free inner loop (vector stores
+// guaranteed by the host); anything else takes the generic loop.
+constexpr int kOutDq = 1, kOutCodes = 2, kOutPacked = 4, kOutSix = 8;
+constexpr int kOutGeneric = -1;
 
 struct TmaParams {
     int32_t ndesc;
@@ -40,10 +53,11 @@ struct TmaParams {
     RowDesc d[kMaxDesc];
 };
 
-// Shared memory after the stages: mbarriers, per-warp top-m lists, per-team
-// radix histograms and broadcast slots.
-constexpr int kTmaExtraBytes = 2 * kTmaMaxStages * 8 + kTmaConsumerWarps * kTopMax * 4 +
-                               kTmaConsumerWarps * 256 * 4 + kTmaConsumerWarps * 4 * 4;
+// Shared memory after the stages: mbarriers, per-warp selection lists,
+// per-slot broadcast records and per-slot radix histograms.
+constexpr int kBcastWords = 8;
+constexpr int kTmaExtraBytes = 2 * kTmaMaxStages * 8 + 2 * kTmaConsumerWarps * kTopMax * 4 +
+                               kTmaConsumerWarps * kBcastWords * 4 + kTmaConsumerWarps * 256 * 4;
 
 // ------------------------------------------------------------- PTX glue --
 
@@ -101,32 +115,20 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
         : "memory");
 }
 
-__device__ __forceinline__ float4 lds_f32x4(uint32_t a) {
-    float4 v;
-    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(a));
-    return v;
-}
-
-__device__ __forceinline__ uint2 lds_u32x2(uint32_t a) {
-    uint2 v;
-    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
-    return v;
-}
-
 // Four consecutive elements (quad j) of a row held in shared memory.
 template <int DT>
 __device__ __forceinline__ void lds_quad(uint32_t row, int j, float v[4]) {
     if constexpr (DT == kF32) {
-        float4 x = lds_f32x4(row + 16u * (uint32_t)j);
-        v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+        asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                     : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3])
+                     : "r"(row + 16u * (uint32_t)j));
     } else {
-        uint2 x = lds_u32x2(row + 8u * (uint32_t)j);
-        v[0] = __uint_as_float(x.x << 16);
-        v[1] = __uint_as_float(x.x & 0xFFFF0000u);
-        v[2] = __uint_as_float(x.y << 16);
-        v[3] = __uint_as_float(x.y & 0xFFFF0000u);
+        uint32_t a, b;
+        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(a), "=r"(b) : "r"(row + 8u * (uint32_t)j));
+        v[0] = __uint_as_float(a << 16);
+        v[1] = __uint_as_float(a & 0xFFFF0000u);
+        v[2] = __uint_as_float(b << 16);
+        v[3] = __uint_as_float(b & 0xFFFF0000u);
     }
 }
 
@@ -134,76 +136,148 @@ __device__ __forceinline__ void named_sync(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-struct Team {
-    int G;        // warps per team
-    int team;     // team index
-    int tw;       // warp index in the team
+// max / min that return NaN when either input is NaN, so a NaN in a row
+// reaches the selected list and is reported as non-finite.
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+    float r;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ float fmin_nan(float a, float b) {
+    float r;
+    asm("min.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+
+// ------------------------------------------------------------------ slot --
+
+// The threads that own one row.
+struct Slot {
+    int lpr;     // threads per row
+    int slot;    // slot index among the consumers
+    int tl;      // thread index within the slot
     int lane;
-    int cw;       // consumer warp index
-    // Named barrier ids never collide between team sizes: a warp may reach
-    // the next tile (another team size) while its old teammates finish.
-    //   G = 2: ids 1..8, G = 4: 9..12, G = 8: 13..14, G = 16: 15.
-    __device__ __forceinline__ void sync() const {
-        if (G == 1) {
-            __syncwarp();
-        } else {
-            const int base = G == 2 ? 1 : G == 4 ? 9 : G == 8 ? 13 : 15;
-            named_sync(base + team, G * 32);
-        }
+    int warp;    // consumer warp index
+    int G;       // warps per row (lpr >= 32), else 1
+    int tw;      // warp index within the slot (lpr >= 32)
+
+    __device__ __forceinline__ void init(int lanes_per_row, int w, int l) {
+        lpr = lanes_per_row;
+        warp = w;
+        lane = l;
+        const int ct = w * 32 + l;
+        slot = ct / lpr;
+        tl = ct % lpr;
+        G = lpr >= 32 ? lpr / 32 : 1;
+        tw = lpr >= 32 ? w % G : 0;
+    }
+    // Named barrier ids never collide between team sizes: after a shape
+    // change every consumer warp meets at barrier 0 first, and within one
+    // shape each team has its own id (G = 2: 1..8, 4: 9..12, 8: 13..14, 16: 15).
+    __device__ __forceinline__ void team_sync() const {
+        const int base = G == 2 ? 1 : G == 4 ? 9 : G == 8 ? 13 : 15;
+        named_sync(base + slot, G * 32);
     }
 };
 
 // ------------------------------------------------------- row selection --
 
+// The M largest of a multiset of |w| (floats >= +0, compared as floats: the
+// same order as their bit patterns), sorted descending (v[0] largest).
+template <int M>
+struct TopMF {
+    float v[M];
+    __device__ __forceinline__ void init() {
+#pragma unroll
+        for (int i = 0; i < M; ++i) v[i] = 0.0f;
+    }
+    __device__ __forceinline__ void insert(float x) {
+#pragma unroll
+        for (int i = 0; i < M; ++i) {
+            const float hi = fmax_nan(v[i], x);
+            if (i + 1 < M) x = fmin_nan(v[i], x);
+            v[i] = hi;
+        }
+    }
+    // union with another sorted list: the (i+1)-th largest of the union is
+    // max(a[i], b[i], max over j < i of min(a[j], b[i-1-j])).
+    __device__ __forceinline__ void merge(const float* b) {
+        float r[M];
+#pragma unroll
+        for (int i = 0; i < M; ++i) {
+            float x = fmax_nan(v[i], b[i]);
+#pragma unroll
+            for (int j = 0; j < i; ++j) x = fmax_nan(x, fmin_nan(v[j], b[i - 1 - j]));
+            r[i] = x;
+        }
+#pragma unroll
+        for (int i = 0; i < M; ++i) v[i] = r[i];
+    }
+    // merge across lanes with xor offsets from `hi` down to 1
+    __device__ __forceinline__ void butterfly(int hi) {
+        for (int off = hi; off >= 1; off >>= 1) {
+            float o[M];
+#pragma unroll
+            for (int i = 0; i < M; ++i) o[i] = __shfl_xor_sync(0xFFFFFFFFu, v[i], off);
+            merge(o);
+        }
+    }
+    // the m-th largest (1 <= m <= M) without a dynamically indexed array
+    __device__ __forceinline__ float get(int m) const {
+        float r = v[0];
+#pragma unroll
+        for (int i = 1; i < M; ++i) r = (m - 1 == i) ? v[i] : r;
+        return r;
+    }
+};
+
+// Per-thread top-M over the quads j = tl, tl + lpr, ... of a row.
 template <int DT, int M>
-__device__ __forceinline__ uint2 tma_select_topm(uint32_t row, int nq, int m, const Team& T,
-                                                 uint32_t* lists) {
-    TopM<M> L;
+__device__ __forceinline__ void topm_scan(uint32_t row, int nq, int tl, int lpr, bool rv, TopMF<M>& L) {
     L.init();
-    for (int j = T.tw * 32 + T.lane; j < nq; j += T.G * 32) {
-        float v[4];
-        lds_quad<DT>(row, j, v);
+    if (!rv) return;
+    int j = tl;
+    for (; j + lpr < nq; j += 2 * lpr) {
+        float a[4], b[4];
+        lds_quad<DT>(row, j, a);
+        lds_quad<DT>(row, j + lpr, b);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) L.insert(abs_key(v[i]));
-    }
-    L.warp_reduce();
-    if (T.G == 1) return make_uint2(L.v[m - 1], L.v[0]);
-    if (T.lane == 0) {
+        for (int i = 0; i < 4; ++i) L.insert(fabsf(a[i]));
 #pragma unroll
-        for (int i = 0; i < M; ++i) lists[T.cw * kTopMax + i] = L.v[i];
+        for (int i = 0; i < 4; ++i) L.insert(fabsf(b[i]));
     }
-    T.sync();
-    TopM<M> R;
-    R.init();
-    const int w0 = T.team * T.G;
-    for (int w = 0; w < T.G; ++w) R.merge(&lists[(w0 + w) * kTopMax]);
-    T.sync();
-    return make_uint2(R.v[m - 1], R.v[0]);
+    if (j < nq) {
+        float a[4];
+        lds_quad<DT>(row, j, a);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) L.insert(fabsf(a[i]));
+    }
 }
 
-// MSB-first radix select (8+8+8+7 bits) over the shared-memory row.
+// MSB-first radix select (8+8+8+7 bits) over the shared-memory row, for a
+// team of G >= 1 whole warps (lpr >= 32).  Sets *nonfinite when a key has an
+// all-ones exponent.
 template <int DT>
-__device__ uint32_t tma_select_radix(uint32_t row, int nq, int64_t m, const Team& T,
-                                     uint32_t* hist, uint32_t* bcast, bool* nonfinite) {
-    const int tt = T.tw * 32 + T.lane;
+__device__ uint32_t select_radix(uint32_t row, int nq, int64_t m, const Slot& T, uint32_t* hist,
+                                 uint32_t* bc, bool* nonfinite) {
     uint32_t prefix = 0, pmask = 0;
     int64_t rem = m;
 #pragma unroll 1
     for (int pass = 0; pass < 4; ++pass) {
         const int shift = pass == 0 ? 23 : pass == 1 ? 15 : pass == 2 ? 7 : 0;
         const uint32_t dmask = pass == 3 ? 0x7Fu : 0xFFu;
-        for (int i = tt; i < 256; i += T.G * 32) hist[i] = 0u;
-        T.sync();
-        for (int j = tt; j < nq; j += T.G * 32) {
+        for (int i = T.tl; i < 256; i += T.lpr) hist[i] = 0u;
+        if (T.G == 1) __syncwarp(); else T.team_sync();
+        for (int j = T.tl; j < nq; j += T.lpr) {
             float v[4];
             lds_quad<DT>(row, j, v);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                uint32_t key = abs_key(v[i]);
+                const uint32_t key = abs_key(v[i]);
                 if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1u);
             }
         }
-        T.sync();
+        if (T.G == 1) __syncwarp(); else T.team_sync();
         if (T.tw == 0) {
             uint32_t cnt[8];
             uint32_t sum = 0;
@@ -215,7 +289,7 @@ __device__ uint32_t tma_select_radix(uint32_t row, int nq, int64_t m, const Team
             uint32_t incl = sum;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
-                uint32_t o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+                const uint32_t o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
                 if (T.lane >= off) incl += o;
             }
             const int64_t excl = (int64_t)(incl - sum);
@@ -224,153 +298,381 @@ __device__ uint32_t tma_select_radix(uint32_t row, int nq, int64_t m, const Team
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     if (acc + cnt[i] >= rem) {
-                        bcast[0] = (uint32_t)(255 - 8 * T.lane - i);
-                        bcast[1] = (uint32_t)(rem - acc);
+                        bc[0] = (uint32_t)(255 - 8 * T.lane - i);
+                        bc[1] = (uint32_t)(rem - acc);
                         break;
                     }
                     acc += cnt[i];
                 }
             }
-            if (pass == 0 && T.lane == 0) bcast[2] = hist[255];
+            if (pass == 0 && T.lane == 0) bc[2] = hist[255];
         }
-        T.sync();
-        const uint32_t b = bcast[0];
-        rem = bcast[1];
-        if (pass == 0) *nonfinite = bcast[2] != 0u;
+        if (T.G == 1) __syncwarp(); else T.team_sync();
+        const uint32_t b = bc[0];
+        rem = bc[1];
+        if (pass == 0) *nonfinite = bc[2] != 0u;
         prefix |= b << shift;
         pmask |= dmask << shift;
-        T.sync();
+        if (T.G == 1) __syncwarp(); else T.team_sync();
     }
     return prefix;
 }
 
-// ---------------------------------------------------- quantize one row --
+// ------------------------------------------------------------ row scale --
 
-// Quantize the four elements of a quad.  b[i] = kMagic + q[i] as a float.
-// FAST: reciprocal product with the near-half guard (warp vote) instead of a
-// division per element; CLIP: clip to [-c, c] first.
-template <bool FAST, bool CLIP>
-__device__ __forceinline__ void quantize_quad(const float v[4], const Scale& S, float b[4]) {
-    float wc[4], y[4], n[4];
-    bool need = false;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        wc[i] = CLIP ? fminf(fmaxf(v[i], -S.c), S.c) : v[i];
-        y[i] = FAST ? __fmul_rn(wc[i], S.rcp) : __fdiv_rn(wc[i], S.s);
-        n[i] = __fsub_rn(__fadd_rn(y[i], kMagic), kMagic);    // rint(y), exact for |y| < 2^22
-        if (FAST) need |= fabsf(__fsub_rn(y[i], n[i])) > kNearHalf;
-    }
-    if (FAST) {
-        if (__any_sync(0xFFFFFFFFu, need)) {
-            if (need) {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    y[i] = __fdiv_rn(wc[i], S.s);
-                    n[i] = __fsub_rn(__fadd_rn(y[i], kMagic), kMagic);
-                }
-            }
-        }
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        float q = fminf(fmaxf(n[i], -S.qmaxf), S.qmaxf);
-        b[i] = S.zero ? kMagic : __fadd_rn(q, kMagic);
+// Everything the quantize loop needs about one row, identical in all the
+// threads of its slot.
+struct RowScale {
+    Scale S;
+    uint32_t hbits;
+    bool range;
+    bool nonfinite;
+    bool clip;     // clip w to [-c, c] before dividing
+    bool clamp;    // clamp the rounded code to [-qmax, qmax]
+};
+
+__device__ __forceinline__ void finish_scale(uint32_t ckey, bool nonfinite, const RowDesc& D, RowScale& R) {
+    uint16_t h;
+    R.S = make_scale(ckey, D.qmax, D.export_mode != 0, &h, &R.range);
+    R.hbits = h;
+    R.nonfinite = nonfinite;
+    // The clip value's own code cq = rint(c / s) is exactly qmax whenever the
+    // scale is a normal number: c / s32 = qmax (1 +- 2^-23), and c / h =
+    // qmax (1 +- 2^-10.9) for a normal binary16 h.  Then the clip can be
+    // skipped (monotone rounded division maps every |w| > c to +-qmax after
+    // the clamp) and, when no |w| exceeds c (m == 1), the clamp too.
+    const bool normal = D.export_mode ? ((h & 0x7C00u) != 0u && (h & 0x7C00u) != 0x7C00u)
+                                      : (R.S.s >= 1.1754943508222875e-38f && R.S.s <= 3.4028234663852886e38f);
+    float cq;
+    if (normal) cq = R.S.qmaxf;
+    else if (R.S.zero) cq = 0.0f;
+    else cq = __fsub_rn(__fadd_rn(__fdiv_rn(R.S.c, R.S.s), kMagic), kMagic);
+    R.clip = !(cq >= R.S.qmaxf);
+    R.clamp = D.m > 1 || !(cq <= R.S.qmaxf);
+}
+
+// Per-row scalar outputs (written by thread 0 of the slot).
+__device__ __forceinline__ void write_row_scalars(const RowDesc& D, int64_t r, const RowScale& R) {
+    const bool per_tensor = D.flags & kPerTensor;
+    if (per_tensor && r != 0) return;
+    const int64_t g = per_tensor ? 0 : r;
+    if (D.clip_out) D.clip_out[g] = R.S.c;
+    if (D.sf32) D.sf32[g] = R.S.s;
+    if (D.sf16) D.sf16[g] = (uint16_t)R.hbits;
+    if (D.status) {
+        const uint32_t st = (R.nonfinite ? kStatusNonfinite : 0u) | (R.range ? kStatusRange : 0u);
+        if (st) atomicOr(reinterpret_cast<unsigned int*>(D.status), st);
     }
 }
 
-template <int DT, bool FAST, bool CLIP>
-__device__ __forceinline__ void tma_quantize_row(const RowDesc& D, int64_t r, uint32_t row, int nq,
-                                                 const Scale& S, const Team& T) {
-    const int64_t n = D.cols;
-    constexpr int esz = DT == kF32 ? 4 : 2;
-    char* dqrow = D.dq ? reinterpret_cast<char*>(D.dq) + r * n * esz : nullptr;
-    int8_t* crow = D.codes ? D.codes + r * n : nullptr;
-    uint8_t* prow = D.packed ? D.packed + r * D.prb : nullptr;
-    const bool vdq = D.flags & kVecDq;
-    const bool vcodes = D.flags & kVecCodes;
-    const bool vpk = D.flags & kVecPacked;
-    const bool six = D.qbits == 6;
-    const int lane = T.lane;
+// ------------------------------------------------------ element kernel --
 
-    for (int jb = T.tw * 32; jb < nq; jb += T.G * 32) {
-        const int j = jb + lane;
-        const bool valid = j < nq;
-        float v[4] = {0.f, 0.f, 0.f, 0.f};
-        if (valid) lds_quad<DT>(row, j, v);
-        float b[4];
-        quantize_quad<FAST, CLIP>(v, S, b);
+// Exact quotients for the lanes where the guard fired (rare); arguments and
+// results travel in registers.
+__device__ __noinline__ float4 exact_round4(float a, float b, float c, float d, float s) {
+    return make_float4(__fsub_rn(__fadd_rn(__fdiv_rn(a, s), kMagic), kMagic),
+                       __fsub_rn(__fadd_rn(__fdiv_rn(b, s), kMagic), kMagic),
+                       __fsub_rn(__fadd_rn(__fdiv_rn(c, s), kMagic), kMagic),
+                       __fsub_rn(__fadd_rn(__fdiv_rn(d, s), kMagic), kMagic));
+}
+
+__device__ __forceinline__ void exact_round8(const float* wc, float s, float* n) {
+    const float4 lo = exact_round4(wc[0], wc[1], wc[2], wc[3], s);
+    const float4 hi = exact_round4(wc[4], wc[5], wc[6], wc[7], s);
+    n[0] = lo.x; n[1] = lo.y; n[2] = lo.z; n[3] = lo.w;
+    n[4] = hi.x; n[5] = hi.y; n[6] = hi.z; n[7] = hi.w;
+}
+
+// Rounded quotients n[i] = rint(fl(wc[i] / s)) of two quads: one reciprocal
+// product each, the exact division only where |y - rint(y)| > 0.5 - 2^-13
+// (see kNearHalf), decided by one warp vote.
+template <bool CLIP>
+__device__ __forceinline__ void round8(const float x[8], const Scale& S, float n[8]) {
+    float wc[8], y[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        wc[i] = CLIP ? fminf(fmaxf(x[i], -S.c), S.c) : x[i];
+        y[i] = __fmul_rn(wc[i], S.rcp);
+        n[i] = __fsub_rn(__fadd_rn(y[i], kMagic), kMagic);
+    }
+    float dmax = fabsf(__fsub_rn(y[0], n[0]));
+#pragma unroll
+    for (int i = 1; i < 8; ++i) dmax = fmaxf(dmax, fabsf(__fsub_rn(y[i], n[i])));
+    const bool need = dmax > kNearHalf;
+    if (__any_sync(0xFFFFFFFFu, need)) {
+        if (need) exact_round8(wc, S.s, n);
+    }
+}
+
+// Stores of one quad for a compile-time output configuration.  b[i] =
+// kMagic + q[i]: its low byte is q's two's-complement byte and its low six
+// bits the int6 field.
+template <int DT, int OUT>
+__device__ __forceinline__ void put_quad(char* dq, int8_t* codes, uint8_t* packed, int j, bool valid, int tl,
+                                         const float q[4], const float b[4], float s) {
+    const uint32_t b0 = __float_as_uint(b[0]), b1 = __float_as_uint(b[1]);
+    const uint32_t b2 = __float_as_uint(b[2]), b3 = __float_as_uint(b[3]);
+    if constexpr ((OUT & kOutDq) != 0) {
+        if (valid) {
+            if constexpr (DT == kF32) {
+                *reinterpret_cast<float4*>(dq + (size_t)j * 16) =
+                    make_float4(__fmul_rn(q[0], s), __fmul_rn(q[1], s), __fmul_rn(q[2], s), __fmul_rn(q[3], s));
+            } else {
+                const uint32_t lo = (uint32_t)float_to_bf16_bits(__fmul_rn(q[0], s)) |
+                                    ((uint32_t)float_to_bf16_bits(__fmul_rn(q[1], s)) << 16);
+                const uint32_t hi = (uint32_t)float_to_bf16_bits(__fmul_rn(q[2], s)) |
+                                    ((uint32_t)float_to_bf16_bits(__fmul_rn(q[3], s)) << 16);
+                *reinterpret_cast<uint2*>(dq + (size_t)j * 8) = make_uint2(lo, hi);
+            }
+        }
+    }
+    if constexpr ((OUT & kOutCodes) != 0 || ((OUT & kOutPacked) != 0 && (OUT & kOutSix) == 0)) {
+        const uint32_t bytes4 = __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
+        if (valid) {
+            if constexpr ((OUT & kOutCodes) != 0) *reinterpret_cast<uint32_t*>(codes + 4 * j) = bytes4;
+            if constexpr ((OUT & kOutPacked) != 0 && (OUT & kOutSix) == 0)
+                *reinterpret_cast<uint32_t*>(packed + 4 * j) = bytes4;
+        }
+    }
+    if constexpr ((OUT & kOutPacked) != 0 && (OUT & kOutSix) != 0) {
+        // four lanes pack 16 codes into three aligned 32-bit words
+        const uint32_t v24 = (b0 & 0x3Fu) | ((b1 << 6) & 0xFC0u) | ((b2 << 12) & 0x3F000u) | ((b3 << 18) & 0xFC0000u);
+        const uint32_t nxt = __shfl_down_sync(0xFFFFFFFFu, v24, 1);
+        const int sub = tl & 3;
+        if (valid && sub < 3)
+            *reinterpret_cast<uint32_t*>(packed + 3 * (j - sub) + 4 * sub) = (v24 >> (8 * sub)) | (nxt << (24 - 8 * sub));
+    }
+}
+
+// Branch-free loop for a common output configuration: reciprocal path, no
+// clip (normal scale), CLAMP when some |w| may exceed c.  All stores are
+// vectorised (the host checked the alignment), all int6 groups are full.
+template <int DT, int OUT, bool CLAMP>
+__device__ __forceinline__ void quantize_row_fast(uint32_t row, int nq, int tl, int lpr, bool rv, float s,
+                                                  float rcp, float qmaxf, char* dq, int8_t* codes,
+                                                  uint8_t* packed) {
+    Scale S;
+    S.c = 0.f;
+    S.s = s;
+    S.rcp = rcp;
+    S.qmaxf = qmaxf;
+    S.fast = true;
+    S.zero = false;
+    const int niter = (nq + lpr - 1) / lpr;
+    int i = 0;
+    for (; i + 1 < niter; i += 2) {
+        const int j0 = tl + lpr * i, j1 = j0 + lpr;
+        const bool v0 = rv, v1 = rv && j1 < nq;
+        float x[8];
+        if (v0) lds_quad<DT>(row, j0, x);
+        else x[0] = x[1] = x[2] = x[3] = 0.f;
+        if (v1) lds_quad<DT>(row, j1, x + 4);
+        else x[4] = x[5] = x[6] = x[7] = 0.f;
+        float n[8];
+        round8<false>(x, S, n);
+        float q[8], b[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            q[k] = CLAMP ? fminf(fmaxf(n[k], -qmaxf), qmaxf) : n[k];
+            b[k] = __fadd_rn(q[k], kMagic);
+        }
+        put_quad<DT, OUT>(dq, codes, packed, j0, v0, tl, q, b, s);
+        put_quad<DT, OUT>(dq, codes, packed, j1, v1, tl, q + 4, b + 4, s);
+    }
+    if (i < niter) {
+        const int j0 = tl + lpr * i;
+        const bool v0 = rv && j0 < nq;
+        float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (v0) lds_quad<DT>(row, j0, x);
+        float n[8];
+        round8<false>(x, S, n);
+        float q[4], b[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            q[k] = CLAMP ? fminf(fmaxf(n[k], -qmaxf), qmaxf) : n[k];
+            b[k] = __fadd_rn(q[k], kMagic);
+        }
+        put_quad<DT, OUT>(dq, codes, packed, j0, v0, tl, q, b, s);
+    }
+}
+
+// Generic loop: any output configuration and alignment, coarse scales (clip),
+// scales outside the reciprocal range (division per element), s == 0.
+template <int DT>
+__device__ __noinline__ void quantize_row_generic(const RowDesc& D, int64_t r, uint32_t row, int nq, int tl,
+                                                  int lpr, bool rv, float c, float s, float rcp, bool fast,
+                                                  bool zero, bool clip, bool clamp) {
+    constexpr int esz = DT == kF32 ? 4 : 2;
+    Scale S;
+    S.c = c;
+    S.s = s;
+    S.rcp = rcp;
+    S.qmaxf = (float)D.qmax;
+    S.fast = fast;
+    S.zero = zero;
+    struct {
+        bool clip, clamp;
+    } R = {clip, clamp};
+    struct {
+        int tl, lpr;
+    } T = {tl, lpr};
+    const int64_t n = D.cols;
+    char* dq = D.dq ? reinterpret_cast<char*>(D.dq) + r * n * esz : nullptr;
+    int8_t* codes = D.codes ? D.codes + r * n : nullptr;
+    uint8_t* packed = D.packed ? D.packed + r * D.prb : nullptr;
+    const bool vdq = D.flags & kVecDq, vcodes = D.flags & kVecCodes, vpk = D.flags & kVecPacked;
+    const bool six = D.qbits == 6;
+    const int niter = (nq + T.lpr - 1) / T.lpr;
+    for (int i = 0; i < niter; ++i) {
+        const int j = T.tl + T.lpr * i;
+        const bool valid = rv && j < nq;
+        float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (valid) lds_quad<DT>(row, j, x);
+        // Rows of one warp may differ in mode (zero scale, reciprocal path,
+        // exact division): every lane computes with per-lane selects so the
+        // warp vote below is reached by all 32 lanes.
+        float wc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        float nn[8];
+        float dmax = 0.0f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            wc[k] = R.clip ? fminf(fmaxf(x[k], -S.c), S.c) : x[k];
+            const float y = S.fast ? __fmul_rn(wc[k], S.rcp) : 0.0f;
+            nn[k] = __fsub_rn(__fadd_rn(y, kMagic), kMagic);
+            dmax = fmaxf(dmax, fabsf(__fsub_rn(y, nn[k])));
+        }
+        const bool need = !S.zero && (!S.fast || dmax > kNearHalf);
+        if (__any_sync(0xFFFFFFFFu, need)) {
+            if (need) exact_round8(wc, S.s, nn);
+        }
+        float q[4], b[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            q[k] = R.clamp ? fminf(fmaxf(nn[k], -S.qmaxf), S.qmaxf) : nn[k];
+            if (S.zero) q[k] = 0.0f;
+            b[k] = __fadd_rn(q[k], kMagic);
+        }
         const int e0 = 4 * j;
-        if (valid && dqrow) {
+        if (valid && dq) {
             float d[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) d[i] = __fmul_rn(__fsub_rn(b[i], kMagic), S.s);
-            if constexpr (DT == kF32) {
-                float* o = reinterpret_cast<float*>(dqrow) + e0;
+            for (int k = 0; k < 4; ++k) d[k] = __fmul_rn(q[k], S.s);
+            if (DT == kF32) {
+                float* o = reinterpret_cast<float*>(dq) + e0;
                 if (vdq) {
                     *reinterpret_cast<float4*>(o) = make_float4(d[0], d[1], d[2], d[3]);
                 } else {
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) o[i] = d[i];
+                    for (int k = 0; k < 4; ++k) o[k] = d[k];
                 }
             } else {
-                uint16_t* o = reinterpret_cast<uint16_t*>(dqrow) + e0;
+                uint16_t* o = reinterpret_cast<uint16_t*>(dq) + e0;
                 uint16_t h[4];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) h[i] = float_to_bf16_bits(d[i]);
+                for (int k = 0; k < 4; ++k) h[k] = float_to_bf16_bits(d[k]);
                 if (vdq) {
                     *reinterpret_cast<uint2*>(o) = make_uint2((uint32_t)h[0] | ((uint32_t)h[1] << 16),
                                                               (uint32_t)h[2] | ((uint32_t)h[3] << 16));
                 } else {
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) o[i] = h[i];
+                    for (int k = 0; k < 4; ++k) o[k] = h[k];
                 }
             }
         }
-        // code bytes: the low byte of kMagic + q is q's two's-complement byte
-        const uint32_t bytes4 = __byte_perm(__byte_perm(__float_as_uint(b[0]), __float_as_uint(b[1]), 0x0040),
-                                            __byte_perm(__float_as_uint(b[2]), __float_as_uint(b[3]), 0x0040),
-                                            0x5410);
-        if (valid && crow) {
+        const uint32_t b0 = __float_as_uint(b[0]), b1 = __float_as_uint(b[1]);
+        const uint32_t b2 = __float_as_uint(b[2]), b3 = __float_as_uint(b[3]);
+        const uint32_t bytes4 = __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
+        if (valid && codes) {
             if (vcodes) {
-                *reinterpret_cast<uint32_t*>(crow + e0) = bytes4;
+                *reinterpret_cast<uint32_t*>(codes + e0) = bytes4;
             } else {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) crow[e0 + i] = (int8_t)(bytes4 >> (8 * i));
+                for (int k = 0; k < 4; ++k) codes[e0 + k] = (int8_t)(bytes4 >> (8 * k));
             }
         }
-        if (prow) {
-            if (six) {
-                const uint32_t v24 = (__float_as_uint(b[0]) & 63u) | ((__float_as_uint(b[1]) & 63u) << 6) |
-                                     ((__float_as_uint(b[2]) & 63u) << 12) | ((__float_as_uint(b[3]) & 63u) << 18);
-                const uint32_t nxt = __shfl_down_sync(0xFFFFFFFFu, v24, 1);
-                const int sub = lane & 3;
-                const int g0 = j - sub;
-                if (valid) {
-                    if (vpk && g0 + 3 < nq) {
-                        if (sub < 3)
-                            *reinterpret_cast<uint32_t*>(prow + 3 * g0 + 4 * sub) =
-                                (v24 >> (8 * sub)) | (nxt << (24 - 8 * sub));
-                    } else {
-                        prow[3 * j + 0] = (uint8_t)(v24 & 0xFFu);
-                        prow[3 * j + 1] = (uint8_t)((v24 >> 8) & 0xFFu);
-                        prow[3 * j + 2] = (uint8_t)((v24 >> 16) & 0xFFu);
-                    }
-                }
-            } else if (valid) {
-                if (vpk) {
-                    *reinterpret_cast<uint32_t*>(prow + e0) = bytes4;
+        if (packed && six) {
+            const uint32_t v24 = (b0 & 0x3Fu) | ((b1 << 6) & 0xFC0u) | ((b2 << 12) & 0x3F000u) | ((b3 << 18) & 0xFC0000u);
+            const uint32_t nxt = __shfl_down_sync(0xFFFFFFFFu, v24, 1);
+            const int sub = T.tl & 3;
+            const int g0 = j - sub;
+            // the group is stored as words only when its four quads exist
+            const bool gfull = g0 + 3 < nq;
+            if (valid) {
+                if (vpk && gfull) {
+                    if (sub < 3)
+                        *reinterpret_cast<uint32_t*>(packed + 3 * g0 + 4 * sub) = (v24 >> (8 * sub)) | (nxt << (24 - 8 * sub));
                 } else {
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) prow[e0 + i] = (uint8_t)(bytes4 >> (8 * i));
+                    packed[3 * j + 0] = (uint8_t)(v24 & 0xFFu);
+                    packed[3 * j + 1] = (uint8_t)((v24 >> 8) & 0xFFu);
+                    packed[3 * j + 2] = (uint8_t)((v24 >> 16) & 0xFFu);
                 }
+            }
+        } else if (packed && valid) {
+            if (vpk) {
+                *reinterpret_cast<uint32_t*>(packed + e0) = bytes4;
+            } else {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) packed[e0 + k] = (uint8_t)(bytes4 >> (8 * k));
             }
         }
     }
 }
 
+template <int DT, int OUT>
+__device__ __forceinline__ void dispatch_fast(bool clamp, uint32_t row, int nq, int tl, int lpr, bool rv,
+                                              const Scale& S, char* dq, int8_t* codes, uint8_t* packed) {
+    if (clamp) quantize_row_fast<DT, OUT, true>(row, nq, tl, lpr, rv, S.s, S.rcp, S.qmaxf, dq, codes, packed);
+    else quantize_row_fast<DT, OUT, false>(row, nq, tl, lpr, rv, S.s, S.rcp, S.qmaxf, dq, codes, packed);
+}
+
+// Quantize + outputs of one row; `rv` false for an idle sub-warp slot (it
+// still takes part in the warp's shuffles and votes).
 template <int DT>
-__device__ __forceinline__ void tma_process_row(const RowDesc& D, int64_t r, uint32_t row, const Team& T,
-                                                uint32_t* lists, uint32_t* hist, uint32_t* bcast) {
+__device__ __forceinline__ void quantize_row(const RowDesc& D, int64_t r, uint32_t row, int nq, const Slot& T,
+                                             bool rv, const RowScale& R) {
+    const int out = D.out_mode;
+    // a warp takes the branch-free loop only if every row it holds can; the
+    // clamp decision must agree too (it is a template parameter there)
+    const bool fast_row = out != kOutGeneric && R.S.fast && !R.S.zero && !R.clip;
+    const bool all_fast = __all_sync(0xFFFFFFFFu, fast_row || !rv);
+    const bool any_clamp = __any_sync(0xFFFFFFFFu, rv && R.clamp);
+    if (!all_fast) {
+        quantize_row_generic<DT>(D, r, row, nq, T.tl, T.lpr, rv, R.S.c, R.S.s, R.S.rcp, R.S.fast, R.S.zero,
+                                 R.clip, R.clamp);
+        return;
+    }
+    constexpr int esz = DT == kF32 ? 4 : 2;
+    char* dq = D.dq ? reinterpret_cast<char*>(D.dq) + r * D.cols * esz : nullptr;
+    int8_t* codes = D.codes ? D.codes + r * D.cols : nullptr;
+    uint8_t* packed = D.packed ? D.packed + r * D.prb : nullptr;
+    switch (out) {
+        case kOutDq | kOutPacked | kOutSix:
+            dispatch_fast<DT, kOutDq | kOutPacked | kOutSix>(any_clamp, row, nq, T.tl, T.lpr, rv, R.S, dq, codes, packed); break;
+        case kOutDq | kOutPacked:
+            dispatch_fast<DT, kOutDq | kOutPacked>(any_clamp, row, nq, T.tl, T.lpr, rv, R.S, dq, codes, packed); break;
+        case kOutDq:
+            dispatch_fast<DT, kOutDq>(any_clamp, row, nq, T.tl, T.lpr, rv, R.S, dq, codes, packed); break;
+        case kOutPacked | kOutSix:
+            dispatch_fast<DT, kOutPacked | kOutSix>(any_clamp, row, nq, T.tl, T.lpr, rv, R.S, dq, codes, packed); break;
+        case kOutPacked:
+            dispatch_fast<DT, kOutPacked>(any_clamp, row, nq, T.tl, T.lpr, rv, R.S, dq, codes, packed); break;
+        case kOutDq | kOutCodes | kOutPacked | kOutSix:
+            dispatch_fast<DT, kOutDq | kOutCodes | kOutPacked | kOutSix>(any_clamp, row, nq, T.tl, T.lpr, rv, R.S, dq, codes, packed); break;
+        case kOutDq | kOutCodes:
+            dispatch_fast<DT, kOutDq | kOutCodes>(any_clamp, row, nq, T.tl, T.lpr, rv, R.S, dq, codes, packed); break;
+        default:
+            quantize_row_generic<DT>(D, r, row, nq, T.tl, T.lpr, rv, R.S.c, R.S.s, R.S.rcp, R.S.fast, R.S.zero,
+                                     R.clip, R.clamp);
+    }
+}
+
+// ---------------------------------------------------------------- rows --
+
+// A row owned by lpr <= 32 threads of one warp (32 / lpr rows per warp).
+// The host routes rows that need the radix select (m > kTopMax) to whole
+// warps, so here m <= kTopMax.
+template <int DT>
+__device__ __forceinline__ void process_row_sub(const RowDesc& D, int64_t r, uint32_t row, const Slot& T, bool rv) {
     const int nq = (int)(D.cols >> 2);
     uint32_t ckey;
     bool nonfinite = false;
@@ -378,42 +680,79 @@ __device__ __forceinline__ void tma_process_row(const RowDesc& D, int64_t r, uin
         ckey = *D.clip_in;
     } else {
         const int m = D.m;
-        uint2 sel;
-        if (m <= 1) sel = tma_select_topm<DT, 1>(row, nq, 1, T, lists);
-        else if (m <= 2) sel = tma_select_topm<DT, 2>(row, nq, m, T, lists);
-        else if (m <= 4) sel = tma_select_topm<DT, 4>(row, nq, m, T, lists);
-        else if (m <= kTopMax) sel = tma_select_topm<DT, 8>(row, nq, m, T, lists);
-        else sel = make_uint2(tma_select_radix<DT>(row, nq, m, T, hist, bcast, &nonfinite), 0u);
-        ckey = sel.x;
-        if (m <= kTopMax) nonfinite = sel.y >= 0x7F800000u;
-    }
-    uint16_t hbits;
-    bool range;
-    const Scale S = make_scale(ckey, D.qmax, D.export_mode != 0, &hbits, &range);
-    const bool per_tensor = D.flags & kPerTensor;
-    if (T.tw == 0 && T.lane == 0 && (!per_tensor || r == 0)) {
-        const int64_t g = per_tensor ? 0 : r;
-        if (D.clip_out) D.clip_out[g] = S.c;
-        if (D.sf32) D.sf32[g] = S.s;
-        if (D.sf16) D.sf16[g] = hbits;
-        if (D.status) {
-            const uint32_t st = (nonfinite ? kStatusNonfinite : 0u) | (range ? kStatusRange : 0u);
-            if (st) atomicOr(reinterpret_cast<unsigned int*>(D.status), st);
+        float sel, top;
+        if (m <= 1) {
+            TopMF<1> L; topm_scan<DT, 1>(row, nq, T.tl, T.lpr, rv, L); L.butterfly(T.lpr >> 1);
+            sel = L.v[0]; top = L.v[0];
+        } else if (m <= 2) {
+            TopMF<2> L; topm_scan<DT, 2>(row, nq, T.tl, T.lpr, rv, L); L.butterfly(T.lpr >> 1);
+            sel = L.get(m); top = L.v[0];
+        } else if (m <= 4) {
+            TopMF<4> L; topm_scan<DT, 4>(row, nq, T.tl, T.lpr, rv, L); L.butterfly(T.lpr >> 1);
+            sel = L.get(m); top = L.v[0];
+        } else {
+            TopMF<8> L; topm_scan<DT, 8>(row, nq, T.tl, T.lpr, rv, L); L.butterfly(T.lpr >> 1);
+            sel = L.get(m); top = L.v[0];
         }
+        ckey = __float_as_uint(sel);
+        nonfinite = !(top <= 3.4028234663852886e38f);
     }
-    if (!(D.flags & kElemOut)) return;
-    // Clipping is a no-op for the codes when the clip value itself rounds to
-    // at least qmax: by monotonicity of rounded division every |w| > c then
-    // also lands on +-qmax after the clamp.  Only coarse (subnormal) scales
-    // need the explicit clip.
-    const float cq = S.zero ? 0.f : __fsub_rn(__fadd_rn(__fdiv_rn(S.c, S.s), kMagic), kMagic);
-    const bool clip = !(cq >= S.qmaxf);
-    if (S.fast && !clip)
-        tma_quantize_row<DT, true, false>(D, r, row, nq, S, T);
-    else if (S.fast)
-        tma_quantize_row<DT, true, true>(D, r, row, nq, S, T);
-    else
-        tma_quantize_row<DT, false, true>(D, r, row, nq, S, T);
+    RowScale R;
+    finish_scale(ckey, nonfinite, D, R);
+    if (rv && T.tl == 0) write_row_scalars(D, r, R);
+    if (D.flags & kElemOut) quantize_row<DT>(D, r, row, nq, T, rv, R);
+}
+
+// Per-warp top-M of a team row, merged by every warp of the team; returns
+// the m-th largest and whether the row holds a non-finite value.  The lists
+// are double-buffered on the parity of the team's row sequence number, so
+// one team barrier per row suffices: a list slot is rewritten two rows
+// later, after a barrier every reader has passed.
+template <int DT, int M>
+__device__ __forceinline__ void team_topm(uint32_t row, int nq, int m, const Slot& T, float* lists, int seq,
+                                          uint32_t* ckey, bool* nonfinite) {
+    TopMF<M> L;
+    topm_scan<DT, M>(row, nq, T.tl, T.lpr, true, L);
+    L.butterfly(16);
+    if (T.G > 1) {
+        float* buf = lists + (seq & 1) * (kTmaConsumerWarps * kTopMax);
+        if (T.lane == 0) {
+#pragma unroll
+            for (int i = 0; i < M; ++i) buf[T.warp * kTopMax + i] = L.v[i];
+        }
+        T.team_sync();
+        L.init();
+        if (T.lane < T.G) {
+            const float* src = buf + (T.slot * T.G + T.lane) * kTopMax;
+#pragma unroll
+            for (int i = 0; i < M; ++i) L.v[i] = src[i];
+        }
+        L.butterfly(T.G >> 1);
+#pragma unroll
+        for (int i = 0; i < M; ++i) L.v[i] = __shfl_sync(0xFFFFFFFFu, L.v[i], 0);
+    }
+    *ckey = __float_as_uint(L.get(m));
+    *nonfinite = !(L.v[0] <= 3.4028234663852886e38f);
+}
+
+// A row owned by G >= 1 whole warps.
+template <int DT>
+__device__ __forceinline__ void process_row_team(const RowDesc& D, int64_t r, uint32_t row, const Slot& T,
+                                                 float* lists, uint32_t* bc, uint32_t* hist, int seq) {
+    const int nq = (int)(D.cols >> 2);
+    const int m = D.m;
+    uint32_t ckey;
+    bool nonfinite = false;
+    if (D.clip_in) ckey = *D.clip_in;
+    else if (m > kTopMax) ckey = select_radix<DT>(row, nq, m, T, hist, bc, &nonfinite);
+    else if (m <= 1) team_topm<DT, 1>(row, nq, 1, T, lists, seq, &ckey, &nonfinite);
+    else if (m <= 2) team_topm<DT, 2>(row, nq, m, T, lists, seq, &ckey, &nonfinite);
+    else if (m <= 4) team_topm<DT, 4>(row, nq, m, T, lists, seq, &ckey, &nonfinite);
+    else team_topm<DT, 8>(row, nq, m, T, lists, seq, &ckey, &nonfinite);
+    RowScale R;
+    finish_scale(ckey, nonfinite, D, R);
+    if (T.tl == 0) write_row_scalars(D, r, R);
+    if (D.flags & kElemOut) quantize_row<DT>(D, r, row, nq, T, true, R);
 }
 
 // ------------------------------------------------------------- kernel --
@@ -426,9 +765,9 @@ rowquant_tma_kernel(const __grid_constant__ TmaParams P) {
     unsigned char* extra = smem + (size_t)S * SB;
     uint64_t* full = reinterpret_cast<uint64_t*>(extra);
     uint64_t* empty = full + kTmaMaxStages;
-    uint32_t* lists = reinterpret_cast<uint32_t*>(empty + kTmaMaxStages);
-    uint32_t* hist = lists + kTmaConsumerWarps * kTopMax;
-    uint32_t* bcast = hist + kTmaConsumerWarps * 256;
+    float* lists = reinterpret_cast<float*>(empty + kTmaMaxStages);                        // [2][warp][kTopMax]
+    uint32_t* bcast = reinterpret_cast<uint32_t*>(lists + 2 * kTmaConsumerWarps * kTopMax);  // [slot][8]
+    uint32_t* hist = bcast + kTmaConsumerWarps * kBcastWords;                          // [slot][256]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -484,33 +823,50 @@ rowquant_tma_kernel(const __grid_constant__ TmaParams P) {
 
     // -------------------------------------------------------- consumers --
     int it = 0;
+    int prev_lpr = 0;
+    int seq = 0;          // rows this warp's team has processed since the last shape change
     for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
         const int s = it % S;
         const int k = it / S;
         const int di = find_desc(P.start, P.ndesc, t);
         const RowDesc& D = P.d[di];
+        const int lpr = D.lanes_per_row;
+        if (lpr != prev_lpr) {
+            // the slot shape changes: no warp may still use the old slots'
+            // shared records (every consumer warp takes this branch on the
+            // same tile)
+            if (prev_lpr != 0) named_sync(0, kTmaConsumers);
+            prev_lpr = lpr;
+            seq = 0;
+        }
         if (!mbar_wait(smem_u32(&full[s]), (uint32_t)(k & 1))) {
             if (lane == 0 && D.status) atomicOr(reinterpret_cast<unsigned int*>(D.status), kStatusTimeout);
             break;
         }
         const int64_t r0 = (t - P.start[di]) * D.tile_rows;
         const int nr = (int)min((int64_t)D.tile_rows, D.rows - r0);
-        const int esz = D.dtype == kF32 ? 4 : 2;
-        const uint32_t row_bytes = (uint32_t)(D.cols * esz);
-        Team T;
-        T.G = D.team_warps;
-        T.cw = warp;
-        T.team = warp / T.G;
-        T.tw = warp % T.G;
-        T.lane = lane;
-        const int teams = kTmaConsumerWarps / T.G;
+        const uint32_t row_bytes = (uint32_t)(D.cols * (D.dtype == kF32 ? 4 : 2));
         const uint32_t stage = smem_base + (uint32_t)s * SB;
-        for (int i = T.team; i < nr; i += teams) {
-            const uint32_t row = stage + (uint32_t)i * row_bytes;
-            if (D.dtype == kF32)
-                tma_process_row<kF32>(D, r0 + i, row, T, lists, hist + T.team * 256, bcast + T.team * 4);
-            else
-                tma_process_row<kBF16>(D, r0 + i, row, T, lists, hist + T.team * 256, bcast + T.team * 4);
+        Slot T;
+        T.init(lpr, warp, lane);
+        const int slots = kTmaConsumers / lpr;
+        if (lpr < 32) {
+            const int rounds = (nr + slots - 1) / slots;
+            for (int rd = 0; rd < rounds; ++rd) {
+                const int i = rd * slots + T.slot;
+                const bool rv = i < nr;
+                const uint32_t row = stage + (uint32_t)(rv ? i : 0) * row_bytes;
+                if (D.dtype == kF32) process_row_sub<kF32>(D, r0 + i, row, T, rv);
+                else process_row_sub<kBF16>(D, r0 + i, row, T, rv);
+            }
+        } else {
+            for (int i = T.slot; i < nr; i += slots, ++seq) {
+                const uint32_t row = stage + (uint32_t)i * row_bytes;
+                uint32_t* bc = bcast + T.slot * kBcastWords;
+                uint32_t* hs = hist + T.slot * 256;
+                if (D.dtype == kF32) process_row_team<kF32>(D, r0 + i, row, T, lists, bc, hs, seq);
+                else process_row_team<kBF16>(D, r0 + i, row, T, lists, bc, hs, seq);
+            }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
