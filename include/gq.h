@@ -250,6 +250,11 @@ GQ_API int64_t gq_k_from_p(int64_t n, double p);
 GQ_API int gq_plan_kind(const char* name, const int64_t* shape, int ndim,
                  int is_float, const char* patterns, int64_t small_numel);
 
+/* The CUDA runtime error code (cudaError_t value) behind the calling
+ * thread's most recent GQ_ERR_CUDA, or 0; and its text from the runtime. */
+GQ_API int gq_last_cuda_error(void);
+GQ_API const char* gq_last_cuda_error_string(void);
+
 /* Static text for a status code. */
 GQ_API const char* gq_status_string(gq_status s);
 

@@ -108,9 +108,16 @@ size_t workspace_size(const gq_tensor* t, int n) {
     return slots * kWsSlot;
 }
 
-gq_status launch_status() {
-    return cudaGetLastError() == cudaSuccess ? GQ_OK : GQ_ERR_CUDA;
+thread_local int g_last_cuda_error = 0;
+
+// GQ_OK, or GQ_ERR_CUDA after recording the CUDA error for gq_last_cuda_error.
+gq_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return GQ_OK;
+    g_last_cuda_error = (int)e;
+    return GQ_ERR_CUDA;
 }
+
+gq_status launch_status() { return cuda_status(cudaGetLastError()); }
 
 // Per-tensor radix select for every per-tensor descriptor (three passes).
 gq_status run_per_tensor_select(const std::vector<SelDesc>& sel, cudaStream_t stream) {
@@ -228,8 +235,8 @@ gq_status run_rows_tma(std::vector<RowDesc>& rows, cudaStream_t stream) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return GQ_ERR_CUDA;
     if (dev >= 0 && dev < kMaxDevices && g_tma_smem_set[dev].load() < (int)smem) {
-        if (cudaFuncSetAttribute(rowquant_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem) != cudaSuccess)
+        if (cuda_status(cudaFuncSetAttribute(rowquant_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem)) != GQ_OK)
             return GQ_ERR_CUDA;
         g_tma_smem_set[dev].store((int)smem);
     }
@@ -292,9 +299,9 @@ gq_status quantize_batch(const gq_tensor* t, int n, Op op, bool f16_mode, void* 
     if (d_status && !aligned(d_status, 4)) return GQ_ERR_MISALIGNED;
     if (n == 0) return GQ_OK;
 
-    if (d_status && cudaMemsetAsync(d_status, 0, sizeof(int32_t) * (size_t)n, stream) != cudaSuccess)
+    if (d_status && cuda_status(cudaMemsetAsync(d_status, 0, sizeof(int32_t) * (size_t)n, stream)) != GQ_OK)
         return GQ_ERR_CUDA;
-    if (need > 0 && cudaMemsetAsync(ws, 0, need, stream) != cudaSuccess) return GQ_ERR_CUDA;
+    if (need > 0 && cuda_status(cudaMemsetAsync(ws, 0, need, stream)) != GQ_OK) return GQ_ERR_CUDA;
 
     std::vector<SelDesc> sel;
     std::vector<RowDesc> rows_w, rows_c;   // warp teams / block teams
@@ -525,6 +532,12 @@ int gq_plan_kind(const char* name, const int64_t* shape, int ndim, int is_float,
         p = comma + 1;
     }
     return GQ_KIND_INT6;
+}
+
+int gq_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* gq_last_cuda_error_string(void) {
+    return g_last_cuda_error ? cudaGetErrorString((cudaError_t)g_last_cuda_error) : "no error";
 }
 
 const char* gq_status_string(gq_status s) {

@@ -136,17 +136,10 @@ __device__ __forceinline__ void named_sync(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-// max / min that return NaN when either input is NaN, so a NaN in a row
-// reaches the selected list and is reported as non-finite.
-__device__ __forceinline__ float fmax_nan(float a, float b) {
-    float r;
-    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
-    return r;
-}
-__device__ __forceinline__ float fmin_nan(float a, float b) {
-    float r;
-    asm("min.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
-    return r;
+// Two floats rounded to bf16 (nearest even), packed low / high.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
 }
 
 // ------------------------------------------------------------------ slot --
@@ -161,15 +154,18 @@ struct Slot {
     int G;       // warps per row (lpr >= 32), else 1
     int tw;      // warp index within the slot (lpr >= 32)
 
+    int lg;      // log2(lpr)
+
     __device__ __forceinline__ void init(int lanes_per_row, int w, int l) {
         lpr = lanes_per_row;
+        lg = 31 - __clz(lpr);
         warp = w;
         lane = l;
         const int ct = w * 32 + l;
-        slot = ct / lpr;
-        tl = ct % lpr;
-        G = lpr >= 32 ? lpr / 32 : 1;
-        tw = lpr >= 32 ? w % G : 0;
+        slot = ct >> lg;
+        tl = ct & (lpr - 1);
+        G = lpr >= 32 ? lpr >> 5 : 1;
+        tw = lpr >= 32 ? (w & (G - 1)) : 0;
     }
     // Named barrier ids never collide between team sizes: after a shape
     // change every consumer warp meets at barrier 0 first, and within one
@@ -184,6 +180,8 @@ struct Slot {
 
 // The M largest of a multiset of |w| (floats >= +0, compared as floats: the
 // same order as their bit patterns), sorted descending (v[0] largest).
+// fmaxf / fminf ignore NaN; topm_scan reports NaN and +-inf separately by
+// forcing v[0] = +inf, which every later merge carries to the top.
 template <int M>
 struct TopMF {
     float v[M];
@@ -194,9 +192,24 @@ struct TopMF {
     __device__ __forceinline__ void insert(float x) {
 #pragma unroll
         for (int i = 0; i < M; ++i) {
-            const float hi = fmax_nan(v[i], x);
-            if (i + 1 < M) x = fmin_nan(v[i], x);
+            const float hi = fmaxf(v[i], x);
+            if (i + 1 < M) x = fminf(v[i], x);
             v[i] = hi;
+        }
+    }
+    // two at a time: for M <= 2 the new top two of {v0 >= v1, a, b} are
+    // max(v0, hi) and max(v1, min(v0, hi), lo) with hi / lo = max / min(a, b)
+    __device__ __forceinline__ void insert2(float a, float b) {
+        if constexpr (M == 1) {
+            v[0] = fmaxf(v[0], fmaxf(a, b));
+        } else if constexpr (M == 2) {
+            const float hi = fmaxf(a, b), lo = fminf(a, b);
+            const float t = fminf(v[0], hi);
+            v[0] = fmaxf(v[0], hi);
+            v[1] = fmaxf(v[1], fmaxf(t, lo));
+        } else {
+            insert(a);
+            insert(b);
         }
     }
     // union with another sorted list: the (i+1)-th largest of the union is
@@ -205,9 +218,9 @@ struct TopMF {
         float r[M];
 #pragma unroll
         for (int i = 0; i < M; ++i) {
-            float x = fmax_nan(v[i], b[i]);
+            float x = fmaxf(v[i], b[i]);
 #pragma unroll
-            for (int j = 0; j < i; ++j) x = fmax_nan(x, fmin_nan(v[j], b[i - 1 - j]));
+            for (int j = 0; j < i; ++j) x = fmaxf(x, fminf(v[j], b[i - 1 - j]));
             r[i] = x;
         }
 #pragma unroll
@@ -231,27 +244,39 @@ struct TopMF {
     }
 };
 
-// Per-thread top-M over the quads j = tl, tl + lpr, ... of a row.
+// Per-thread top-M over the quads j = tl, tl + lpr, ... of a row.  bad
+// accumulates x * 0, which is NaN exactly when some x is NaN or +-inf.
 template <int DT, int M>
-__device__ __forceinline__ void topm_scan(uint32_t row, int nq, int tl, int lpr, bool rv, TopMF<M>& L) {
+__device__ __forceinline__ void topm_scan(uint32_t row, int nq, int tl, int lpr, int lg, bool rv, TopMF<M>& L) {
+    constexpr uint32_t QB = DT == kF32 ? 16u : 8u;       // bytes of a quad in shared memory
     L.init();
     if (!rv) return;
-    int j = tl;
-    for (; j + lpr < nq; j += 2 * lpr) {
+    float bad = 0.0f;
+    const int nfull = nq >> lg;                           // quads every thread of the slot has
+    const uint32_t step = QB * (uint32_t)lpr;
+    uint32_t sa = row + QB * (uint32_t)tl;
+    int i = 0;
+    for (; i + 2 <= nfull; i += 2, sa += 2 * step) {
         float a[4], b[4];
-        lds_quad<DT>(row, j, a);
-        lds_quad<DT>(row, j + lpr, b);
+        lds_quad<DT>(sa, 0, a);
+        lds_quad<DT>(sa + step, 0, b);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) L.insert(fabsf(a[i]));
-#pragma unroll
-        for (int i = 0; i < 4; ++i) L.insert(fabsf(b[i]));
+        for (int k = 0; k < 4; ++k) {
+            L.insert2(fabsf(a[k]), fabsf(b[k]));
+            bad = __fmaf_rn(a[k], 0.0f, bad);
+            bad = __fmaf_rn(b[k], 0.0f, bad);
+        }
     }
-    if (j < nq) {
+    for (int j = tl + lpr * i; j < nq; j += lpr, sa += step) {
         float a[4];
-        lds_quad<DT>(row, j, a);
+        lds_quad<DT>(sa, 0, a);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) L.insert(fabsf(a[i]));
+        for (int k = 0; k < 4; ++k) {
+            L.insert(fabsf(a[k]));
+            bad = __fmaf_rn(a[k], 0.0f, bad);
+        }
     }
+    if (bad != bad) L.v[0] = __int_as_float(0x7F800000);   // +inf marks a non-finite row
 }
 
 // MSB-first radix select (8+8+8+7 bits) over the shared-memory row, for a
@@ -404,53 +429,57 @@ __device__ __forceinline__ void round8(const float x[8], const Scale& S, float n
     }
 }
 
-// Stores of one quad for a compile-time output configuration.  b[i] =
-// kMagic + q[i]: its low byte is q's two's-complement byte and its low six
-// bits the int6 field.
+// Stores of one quad for a compile-time output configuration, at running
+// pointers: pd (w_hat quad), pc (4 code bytes), pp (int8: 4 bytes; int6: this
+// lane's 32-bit word of its 4-lane group, unused by the group's 4th lane).
+// b[i] = kMagic + q[i]: its low byte is q's two's-complement byte and its low
+// six bits the int6 field.
 template <int DT, int OUT>
-__device__ __forceinline__ void put_quad(char* dq, int8_t* codes, uint8_t* packed, int j, bool valid, int tl,
+__device__ __forceinline__ void put_quad(char* pd, int8_t* pc, uint8_t* pp, bool valid, int sub,
                                          const float q[4], const float b[4], float s) {
     const uint32_t b0 = __float_as_uint(b[0]), b1 = __float_as_uint(b[1]);
     const uint32_t b2 = __float_as_uint(b[2]), b3 = __float_as_uint(b[3]);
     if constexpr ((OUT & kOutDq) != 0) {
-        if (valid) {
-            if constexpr (DT == kF32) {
-                *reinterpret_cast<float4*>(dq + (size_t)j * 16) =
-                    make_float4(__fmul_rn(q[0], s), __fmul_rn(q[1], s), __fmul_rn(q[2], s), __fmul_rn(q[3], s));
-            } else {
-                const uint32_t lo = (uint32_t)float_to_bf16_bits(__fmul_rn(q[0], s)) |
-                                    ((uint32_t)float_to_bf16_bits(__fmul_rn(q[1], s)) << 16);
-                const uint32_t hi = (uint32_t)float_to_bf16_bits(__fmul_rn(q[2], s)) |
-                                    ((uint32_t)float_to_bf16_bits(__fmul_rn(q[3], s)) << 16);
-                *reinterpret_cast<uint2*>(dq + (size_t)j * 8) = make_uint2(lo, hi);
-            }
+        if constexpr (DT == kF32) {
+            const float4 d = make_float4(__fmul_rn(q[0], s), __fmul_rn(q[1], s), __fmul_rn(q[2], s), __fmul_rn(q[3], s));
+            if (valid) *reinterpret_cast<float4*>(pd) = d;
+        } else {
+            const uint2 d = make_uint2(pack_bf16x2(__fmul_rn(q[0], s), __fmul_rn(q[1], s)),
+                                       pack_bf16x2(__fmul_rn(q[2], s), __fmul_rn(q[3], s)));
+            if (valid) *reinterpret_cast<uint2*>(pd) = d;
         }
     }
     if constexpr ((OUT & kOutCodes) != 0 || ((OUT & kOutPacked) != 0 && (OUT & kOutSix) == 0)) {
         const uint32_t bytes4 = __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
-        if (valid) {
-            if constexpr ((OUT & kOutCodes) != 0) *reinterpret_cast<uint32_t*>(codes + 4 * j) = bytes4;
-            if constexpr ((OUT & kOutPacked) != 0 && (OUT & kOutSix) == 0)
-                *reinterpret_cast<uint32_t*>(packed + 4 * j) = bytes4;
+        if constexpr ((OUT & kOutCodes) != 0) {
+            if (valid) *reinterpret_cast<uint32_t*>(pc) = bytes4;
+        }
+        if constexpr ((OUT & kOutPacked) != 0 && (OUT & kOutSix) == 0) {
+            if (valid) *reinterpret_cast<uint32_t*>(pp) = bytes4;
         }
     }
     if constexpr ((OUT & kOutPacked) != 0 && (OUT & kOutSix) != 0) {
         // four lanes pack 16 codes into three aligned 32-bit words
         const uint32_t v24 = (b0 & 0x3Fu) | ((b1 << 6) & 0xFC0u) | ((b2 << 12) & 0x3F000u) | ((b3 << 18) & 0xFC0000u);
         const uint32_t nxt = __shfl_down_sync(0xFFFFFFFFu, v24, 1);
-        const int sub = tl & 3;
-        if (valid && sub < 3)
-            *reinterpret_cast<uint32_t*>(packed + 3 * (j - sub) + 4 * sub) = (v24 >> (8 * sub)) | (nxt << (24 - 8 * sub));
+        const uint32_t word = (v24 >> (8 * sub)) | (nxt << (24 - 8 * sub));
+        if (valid && sub < 3) *reinterpret_cast<uint32_t*>(pp) = word;
     }
 }
 
 // Branch-free loop for a common output configuration: reciprocal path, no
 // clip (normal scale), CLAMP when some |w| may exceed c.  All stores are
 // vectorised (the host checked the alignment), all int6 groups are full.
+// Full trips (two quads every thread of the slot has) run without any
+// per-lane test; stores are predicated on rv (an idle sub-warp slot reads a
+// valid row and writes nothing).
 template <int DT, int OUT, bool CLAMP>
-__device__ __forceinline__ void quantize_row_fast(uint32_t row, int nq, int tl, int lpr, bool rv, float s,
-                                                  float rcp, float qmaxf, char* dq, int8_t* codes,
+__device__ __forceinline__ void quantize_row_fast(uint32_t row, int nq, int tl, int lpr, int lg, bool rv,
+                                                  float s, float rcp, float qmaxf, char* dq, int8_t* codes,
                                                   uint8_t* packed) {
+    constexpr uint32_t QB = DT == kF32 ? 16u : 8u;
+    constexpr int DQB = DT == kF32 ? 16 : 8;
+    constexpr bool SIX = (OUT & kOutSix) != 0;
     Scale S;
     S.c = 0.f;
     S.s = s;
@@ -458,32 +487,49 @@ __device__ __forceinline__ void quantize_row_fast(uint32_t row, int nq, int tl, 
     S.qmaxf = qmaxf;
     S.fast = true;
     S.zero = false;
-    const int niter = (nq + lpr - 1) / lpr;
+    const int sub = tl & 3;
+    const uint32_t step = QB * (uint32_t)lpr;
+    uint32_t sa = row + QB * (uint32_t)tl;
+    char* pd = dq + DQB * tl;
+    int8_t* pc = codes + 4 * tl;
+    uint8_t* pp = packed + (SIX ? 3 * (tl - sub) + 4 * sub : 4 * tl);
+    const int sd = DQB * lpr, sc = 4 * lpr, sp = SIX ? 3 * lpr : 4 * lpr;
+    const int nfull = nq >> lg;
     int i = 0;
-    for (; i + 1 < niter; i += 2) {
-        const int j0 = tl + lpr * i, j1 = j0 + lpr;
-        const bool v0 = rv, v1 = rv && j1 < nq;
+    for (; i + 2 <= nfull; i += 2) {
         float x[8];
-        if (v0) lds_quad<DT>(row, j0, x);
-        else x[0] = x[1] = x[2] = x[3] = 0.f;
-        if (v1) lds_quad<DT>(row, j1, x + 4);
-        else x[4] = x[5] = x[6] = x[7] = 0.f;
+        lds_quad<DT>(sa, 0, x);
+        lds_quad<DT>(sa + step, 0, x + 4);
         float n[8];
         round8<false>(x, S, n);
         float q[8], b[8];
+        if (CLAMP) {
+            // only codes of |w| > c can exceed qmax: clamp when the warp has one
+            float nmax = fabsf(n[0]);
+#pragma unroll
+            for (int k = 1; k < 8; ++k) nmax = fmaxf(nmax, fabsf(n[k]));
+            if (__any_sync(0xFFFFFFFFu, nmax > qmaxf)) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) n[k] = fminf(fmaxf(n[k], -qmaxf), qmaxf);
+            }
+        }
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-            q[k] = CLAMP ? fminf(fmaxf(n[k], -qmaxf), qmaxf) : n[k];
+            q[k] = n[k];
             b[k] = __fadd_rn(q[k], kMagic);
         }
-        put_quad<DT, OUT>(dq, codes, packed, j0, v0, tl, q, b, s);
-        put_quad<DT, OUT>(dq, codes, packed, j1, v1, tl, q + 4, b + 4, s);
+        put_quad<DT, OUT>(pd, pc, pp, rv, sub, q, b, s);
+        put_quad<DT, OUT>(pd + sd, pc + sc, pp + sp, rv, sub, q + 4, b + 4, s);
+        sa += 2 * step;
+        pd += 2 * sd;
+        pc += 2 * sc;
+        pp += 2 * sp;
     }
-    if (i < niter) {
-        const int j0 = tl + lpr * i;
-        const bool v0 = rv && j0 < nq;
+    const int niter = (nq + lpr - 1) >> lg;
+    for (; i < niter; ++i) {
+        const bool valid = rv && (tl + lpr * i < nq);
         float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        if (v0) lds_quad<DT>(row, j0, x);
+        if (valid) lds_quad<DT>(sa, 0, x);
         float n[8];
         round8<false>(x, S, n);
         float q[4], b[4];
@@ -492,22 +538,26 @@ __device__ __forceinline__ void quantize_row_fast(uint32_t row, int nq, int tl, 
             q[k] = CLAMP ? fminf(fmaxf(n[k], -qmaxf), qmaxf) : n[k];
             b[k] = __fadd_rn(q[k], kMagic);
         }
-        put_quad<DT, OUT>(dq, codes, packed, j0, v0, tl, q, b, s);
+        put_quad<DT, OUT>(pd, pc, pp, valid, sub, q, b, s);
+        sa += step;
+        pd += sd;
+        pc += sc;
+        pp += sp;
     }
 }
 
 // Generic loop: any output configuration and alignment, coarse scales (clip),
 // scales outside the reciprocal range (division per element), s == 0.
 template <int DT>
-__device__ __noinline__ void quantize_row_generic(const RowDesc& D, int64_t r, uint32_t row, int nq, int tl,
-                                                  int lpr, bool rv, float c, float s, float rcp, bool fast,
-                                                  bool zero, bool clip, bool clamp) {
-    constexpr int esz = DT == kF32 ? 4 : 2;
+__device__ __forceinline__ void quantize_row_generic(uint32_t row, int nq, int tl, int lpr, bool rv, float c,
+                                                  float s, float rcp, float qmaxf, bool fast, bool zero,
+                                                  bool clip, bool clamp, char* dq, int8_t* codes,
+                                                  uint8_t* packed, bool vdq, bool vcodes, bool vpk, bool six) {
     Scale S;
     S.c = c;
     S.s = s;
     S.rcp = rcp;
-    S.qmaxf = (float)D.qmax;
+    S.qmaxf = qmaxf;
     S.fast = fast;
     S.zero = zero;
     struct {
@@ -516,13 +566,7 @@ __device__ __noinline__ void quantize_row_generic(const RowDesc& D, int64_t r, u
     struct {
         int tl, lpr;
     } T = {tl, lpr};
-    const int64_t n = D.cols;
-    char* dq = D.dq ? reinterpret_cast<char*>(D.dq) + r * n * esz : nullptr;
-    int8_t* codes = D.codes ? D.codes + r * n : nullptr;
-    uint8_t* packed = D.packed ? D.packed + r * D.prb : nullptr;
-    const bool vdq = D.flags & kVecDq, vcodes = D.flags & kVecCodes, vpk = D.flags & kVecPacked;
-    const bool six = D.qbits == 6;
-    const int niter = (nq + T.lpr - 1) / T.lpr;
+    const int niter = (nq + T.lpr - 1) >> (31 - __clz(T.lpr));
     for (int i = 0; i < niter; ++i) {
         const int j = T.tl + T.lpr * i;
         const bool valid = rv && j < nq;
@@ -621,8 +665,9 @@ __device__ __noinline__ void quantize_row_generic(const RowDesc& D, int64_t r, u
 template <int DT, int OUT>
 __device__ __forceinline__ void dispatch_fast(bool clamp, uint32_t row, int nq, int tl, int lpr, bool rv,
                                               const Scale& S, char* dq, int8_t* codes, uint8_t* packed) {
-    if (clamp) quantize_row_fast<DT, OUT, true>(row, nq, tl, lpr, rv, S.s, S.rcp, S.qmaxf, dq, codes, packed);
-    else quantize_row_fast<DT, OUT, false>(row, nq, tl, lpr, rv, S.s, S.rcp, S.qmaxf, dq, codes, packed);
+    const int lg = 31 - __clz(lpr);
+    if (clamp) quantize_row_fast<DT, OUT, true>(row, nq, tl, lpr, lg, rv, S.s, S.rcp, S.qmaxf, dq, codes, packed);
+    else quantize_row_fast<DT, OUT, false>(row, nq, tl, lpr, lg, rv, S.s, S.rcp, S.qmaxf, dq, codes, packed);
 }
 
 // Quantize + outputs of one row; `rv` false for an idle sub-warp slot (it
@@ -631,20 +676,21 @@ template <int DT>
 __device__ __forceinline__ void quantize_row(const RowDesc& D, int64_t r, uint32_t row, int nq, const Slot& T,
                                              bool rv, const RowScale& R) {
     const int out = D.out_mode;
+    constexpr int esz = DT == kF32 ? 4 : 2;
+    char* dq = D.dq ? reinterpret_cast<char*>(D.dq) + r * D.cols * esz : nullptr;
+    int8_t* codes = D.codes ? D.codes + r * D.cols : nullptr;
+    uint8_t* packed = D.packed ? D.packed + r * D.prb : nullptr;
     // a warp takes the branch-free loop only if every row it holds can; the
     // clamp decision must agree too (it is a template parameter there)
     const bool fast_row = out != kOutGeneric && R.S.fast && !R.S.zero && !R.clip;
     const bool all_fast = __all_sync(0xFFFFFFFFu, fast_row || !rv);
     const bool any_clamp = __any_sync(0xFFFFFFFFu, rv && R.clamp);
     if (!all_fast) {
-        quantize_row_generic<DT>(D, r, row, nq, T.tl, T.lpr, rv, R.S.c, R.S.s, R.S.rcp, R.S.fast, R.S.zero,
-                                 R.clip, R.clamp);
+        quantize_row_generic<DT>(row, nq, T.tl, T.lpr, rv, R.S.c, R.S.s, R.S.rcp, R.S.qmaxf, R.S.fast, R.S.zero,
+                                 R.clip, R.clamp, dq, codes, packed, (D.flags & kVecDq) != 0,
+                                 (D.flags & kVecCodes) != 0, (D.flags & kVecPacked) != 0, D.qbits == 6);
         return;
     }
-    constexpr int esz = DT == kF32 ? 4 : 2;
-    char* dq = D.dq ? reinterpret_cast<char*>(D.dq) + r * D.cols * esz : nullptr;
-    int8_t* codes = D.codes ? D.codes + r * D.cols : nullptr;
-    uint8_t* packed = D.packed ? D.packed + r * D.prb : nullptr;
     switch (out) {
         case kOutDq | kOutPacked | kOutSix:
             dispatch_fast<DT, kOutDq | kOutPacked | kOutSix>(any_clamp, row, nq, T.tl, T.lpr, rv, R.S, dq, codes, packed); break;
@@ -658,11 +704,8 @@ __device__ __forceinline__ void quantize_row(const RowDesc& D, int64_t r, uint32
             dispatch_fast<DT, kOutPacked>(any_clamp, row, nq, T.tl, T.lpr, rv, R.S, dq, codes, packed); break;
         case kOutDq | kOutCodes | kOutPacked | kOutSix:
             dispatch_fast<DT, kOutDq | kOutCodes | kOutPacked | kOutSix>(any_clamp, row, nq, T.tl, T.lpr, rv, R.S, dq, codes, packed); break;
-        case kOutDq | kOutCodes:
-            dispatch_fast<DT, kOutDq | kOutCodes>(any_clamp, row, nq, T.tl, T.lpr, rv, R.S, dq, codes, packed); break;
         default:
-            quantize_row_generic<DT>(D, r, row, nq, T.tl, T.lpr, rv, R.S.c, R.S.s, R.S.rcp, R.S.fast, R.S.zero,
-                                     R.clip, R.clamp);
+            dispatch_fast<DT, kOutDq | kOutCodes>(any_clamp, row, nq, T.tl, T.lpr, rv, R.S, dq, codes, packed); break;
     }
 }
 
@@ -682,16 +725,16 @@ __device__ __forceinline__ void process_row_sub(const RowDesc& D, int64_t r, uin
         const int m = D.m;
         float sel, top;
         if (m <= 1) {
-            TopMF<1> L; topm_scan<DT, 1>(row, nq, T.tl, T.lpr, rv, L); L.butterfly(T.lpr >> 1);
+            TopMF<1> L; topm_scan<DT, 1>(row, nq, T.tl, T.lpr, T.lg, rv, L); L.butterfly(T.lpr >> 1);
             sel = L.v[0]; top = L.v[0];
         } else if (m <= 2) {
-            TopMF<2> L; topm_scan<DT, 2>(row, nq, T.tl, T.lpr, rv, L); L.butterfly(T.lpr >> 1);
+            TopMF<2> L; topm_scan<DT, 2>(row, nq, T.tl, T.lpr, T.lg, rv, L); L.butterfly(T.lpr >> 1);
             sel = L.get(m); top = L.v[0];
         } else if (m <= 4) {
-            TopMF<4> L; topm_scan<DT, 4>(row, nq, T.tl, T.lpr, rv, L); L.butterfly(T.lpr >> 1);
+            TopMF<4> L; topm_scan<DT, 4>(row, nq, T.tl, T.lpr, T.lg, rv, L); L.butterfly(T.lpr >> 1);
             sel = L.get(m); top = L.v[0];
         } else {
-            TopMF<8> L; topm_scan<DT, 8>(row, nq, T.tl, T.lpr, rv, L); L.butterfly(T.lpr >> 1);
+            TopMF<8> L; topm_scan<DT, 8>(row, nq, T.tl, T.lpr, T.lg, rv, L); L.butterfly(T.lpr >> 1);
             sel = L.get(m); top = L.v[0];
         }
         ckey = __float_as_uint(sel);
@@ -712,7 +755,7 @@ template <int DT, int M>
 __device__ __forceinline__ void team_topm(uint32_t row, int nq, int m, const Slot& T, float* lists, int seq,
                                           uint32_t* ckey, bool* nonfinite) {
     TopMF<M> L;
-    topm_scan<DT, M>(row, nq, T.tl, T.lpr, true, L);
+    topm_scan<DT, M>(row, nq, T.tl, T.lpr, T.lg, true, L);
     L.butterfly(16);
     if (T.G > 1) {
         float* buf = lists + (seq & 1) * (kTmaConsumerWarps * kTopMax);
@@ -849,7 +892,7 @@ rowquant_tma_kernel(const __grid_constant__ TmaParams P) {
         const uint32_t stage = smem_base + (uint32_t)s * SB;
         Slot T;
         T.init(lpr, warp, lane);
-        const int slots = kTmaConsumers / lpr;
+        const int slots = kTmaConsumers >> T.lg;
         if (lpr < 32) {
             const int rounds = (nr + slots - 1) / slots;
             for (int rd = 0; rd < rounds; ++rd) {

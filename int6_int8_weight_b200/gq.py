@@ -39,12 +39,12 @@ STATUS_NAMES = {0: "GQ_OK", 1: "GQ_ERR_INVALID_ARG", 2: "GQ_ERR_UNSUPPORTED",
 
 EXPORTED = ("gq_row_clip_select", "gq_fakequant_fwd", "gq_ste_bwd", "gq_export_pack",
             "gq_export_pack_noalloc", "gq_dequant", "gq_workspace_size", "gq_packed_row_bytes", "gq_k_from_p",
-            "gq_plan_kind", "gq_status_string")
+            "gq_plan_kind", "gq_status_string", "gq_last_cuda_error", "gq_last_cuda_error_string")
 
 
 class GQError(RuntimeError):
-    def __init__(self, status: int, where: str):
-        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+    def __init__(self, status: int, where: str, detail: str = ""):
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}" + (f" ({detail})" if detail else ""))
         self.status = status
 
 
@@ -86,6 +86,10 @@ def _load() -> C.CDLL:
     L.gq_plan_kind.restype = i32
     L.gq_status_string.argtypes = [i32]
     L.gq_status_string.restype = C.c_char_p
+    L.gq_last_cuda_error.argtypes = []
+    L.gq_last_cuda_error.restype = i32
+    L.gq_last_cuda_error_string.argtypes = []
+    L.gq_last_cuda_error_string.restype = C.c_char_p
     return L
 
 
@@ -102,7 +106,8 @@ def _stream(stream) -> int | None:
 
 def _check(status: int, where: str):
     if status != GQ_OK:
-        raise GQError(status, where)
+        detail = LIB.gq_last_cuda_error_string().decode() if status == 7 else ""
+        raise GQError(status, where, detail)
 
 
 def _arr(descs):
