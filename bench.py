@@ -122,7 +122,7 @@ def kernel_source_hash():
 
 
 def traffic_per_launch(kernel_hash):
-    """ncu DRAM bytes per launch of the fused pass, if taken on this source."""
+    """ncu DRAM bytes of one step's fused launches, if taken on this source."""
     path = os.path.join(ROOT, "profiles", "rowquant_traffic.json")
     try:
         with open(path) as f:
@@ -438,10 +438,13 @@ def run_ours(args, world, rank, local):
             per_call[i] += dt
             launch_s += dt
     achieved = wl.alg_bytes * args.steps / launch_s / 1e9
-    traffic, tinfo = traffic_per_launch(kernel_source_hash())
+    traffic_step, tinfo = traffic_per_launch(kernel_source_hash())
+    traffic = None
+    if traffic_step is not None and tinfo.get("launches_per_step") == ncalls and not args.only:
+        traffic = int(traffic_step / ncalls)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "peak_source": peak_kind,
-                "traffic": traffic,
+                "traffic": traffic, "algorithmic_bytes_per_launch": int(wl.alg_bytes / ncalls),
                 "kernel": "rowquant_kernel (fused clip-select + quantize + dequant + pack), all "
                           f"{ncalls} launches of a step",
                 "algorithmic_bytes_per_step": wl.alg_bytes,

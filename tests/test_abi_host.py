@@ -158,3 +158,8 @@ def test_other_argument_errors(gq):
     assert L.gq_dequant(None, None, 6, 0, 0, 4, None, 0, None) == 0  # empty is a no-op
     # empty batch is a no-op
     assert L.gq_export_pack(gq._arr([]), 0, None, 0, None, None) == 0
+
+
+def test_last_cuda_error_starts_clear(gq):
+    assert gq.LIB.gq_last_cuda_error() == 0
+    assert gq.LIB.gq_last_cuda_error_string().decode() == "no error"
