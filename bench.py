@@ -110,14 +110,17 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+FUSED_KERNEL_SOURCES = ("gq_device.cuh", "gq_kernels.cuh", "gq_rowquant_tma.cuh")
+
+
 def kernel_source_hash():
+    """Hash of the sources the fused per-row kernel is built from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "int6_int8_weight_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode())
-                h.update(f.read())
+    for name in FUSED_KERNEL_SOURCES:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 

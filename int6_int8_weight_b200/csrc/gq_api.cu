@@ -11,6 +11,7 @@
 #include <vector>
 
 #include "gq.h"
+#include "gq_aux_kernels.cuh"
 #include "gq_kernels.cuh"
 #include "gq_rowquant_tma.cuh"
 
@@ -482,13 +483,14 @@ gq_status gq_dequant(const uint8_t* d_packed, const uint16_t* d_scale_f16, int q
     const size_t esz = out_dtype == GQ_F32 ? 4 : 2;
     if (!aligned(d_scale_f16, 2) || !aligned(d_out, esz)) return GQ_ERR_MISALIGNED;
     const int64_t prb = packed_row_bytes(cols, qbits);
-    const int vec_out = out_dtype == GQ_F32 && aligned(d_out, 16) && (cols % 4) == 0;
-    const int64_t total = rows * ((cols + 3) / 4);
+    const size_t vin = out_dtype == GQ_F32 ? 16 : 8;
+    const int vec_out = aligned(d_out, vin) && ((cols * (int64_t)esz) % (int64_t)vin) == 0;
+    const int words = aligned(d_packed, 4) && (qbits == 6 ? (cols % 16) == 0 : (cols % 4) == 0);
     const int64_t blocks = std::min<int64_t>((int64_t)sm_count() * 8,
-                                             (total + kBlockThreads - 1) / kBlockThreads);
+                                             (rows + kBlockWarps - 1) / kBlockWarps);
     dequant_kernel<<<(unsigned)blocks, kBlockThreads, 0, stream>>>(
         d_packed, d_scale_f16, qbits, gran == GQ_PER_TENSOR, rows, cols, prb, d_out, out_dtype,
-        vec_out);
+        vec_out, words);
     return launch_status();
 }
 

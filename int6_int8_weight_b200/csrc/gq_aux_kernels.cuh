@@ -1,0 +1,322 @@
+// gq_aux_kernels.cuh -- the kernels around the fused per-row pass:
+//  ptsel_kernel<PASS>    per-tensor radix select, three histogram passes
+//                        (11 + 11 + 9 bits of |w|); the last block of each
+//                        tensor picks the bucket (ticket counter, no spin).
+//  ste_kernel            straight-through backward: copy or accumulate.
+//  dequant_kernel        dequant on load from packed codes + binary16 scales.
+//  passthrough_kernel    binary16 round-to-nearest-even of small tensors.
+#pragma once
+
+#include "gq_kernels.cuh"
+
+namespace gq {
+
+// ------------------------------------------------- per-tensor selection --
+
+struct SelDesc {
+    const void* w;
+    uint32_t* hist;            // 2048 counters in the workspace
+    uint32_t* state;           // [0] prefix [1] remaining [2] ticket [3] key
+    int32_t* status;
+    int64_t rows, cols, ld;
+    int64_t rows_per_item;
+    int64_t items;
+    int64_t m;
+    int32_t dtype;
+    int32_t pad;
+};
+
+struct SelParams {
+    int32_t ndesc;
+    int32_t pad;
+    int64_t start[kMaxDesc + 1];
+    SelDesc d[kMaxDesc];
+};
+
+constexpr int kSelBins = 2048;
+
+// PASS 0: digit = key bits 30..20; PASS 1: bits 19..9 among keys whose bits
+// 30..20 equal the chosen prefix; PASS 2: bits 8..0 among keys whose bits
+// 30..9 match.  One block per item (a block of rows of one tensor).
+template <int PASS>
+__global__ void __launch_bounds__(kBlockThreads)
+ptsel_kernel(const __grid_constant__ SelParams P) {
+    __shared__ uint32_t h[kSelBins];
+    __shared__ uint32_t s_warp[kBlockWarps];
+    __shared__ int s_last;
+    const int tid = threadIdx.x;
+    const int64_t item = blockIdx.x;
+    const int di = find_desc(P.start, P.ndesc, item);
+    const SelDesc& D = P.d[di];
+    const int64_t it = item - P.start[di];
+
+    for (int i = tid; i < kSelBins; i += kBlockThreads) h[i] = 0u;
+    __syncthreads();
+
+    const uint32_t prefix = PASS == 0 ? 0u : __ldcg(&D.state[0]);
+    const int64_t r0 = it * D.rows_per_item;
+    const int64_t r1 = min(D.rows, r0 + D.rows_per_item);
+    const int esz = D.dtype == kF32 ? 4 : 2;
+    bool bad = false;
+    auto count = [&](float x) {
+        const uint32_t key = abs_key(x);
+        if (PASS == 0) {
+            bad |= key >= 0x7F800000u;
+            atomicAdd(&h[key >> 20], 1u);
+        } else if (PASS == 1) {
+            if ((key >> 20) == prefix) atomicAdd(&h[(key >> 9) & 0x7FFu], 1u);
+        } else {
+            if ((key >> 9) == prefix) atomicAdd(&h[key & 0x1FFu], 1u);
+        }
+    };
+    const bool flat = D.ld == D.cols;
+    const bool vec = flat && D.dtype == kF32 && (reinterpret_cast<uintptr_t>(D.w) & 15u) == 0 &&
+                     ((r0 * D.cols) & 3) == 0;
+    if (vec) {
+        // contiguous fp32 rows, 16-byte aligned: four elements per thread and step
+        const int64_t e0 = r0 * D.cols, e1 = r1 * D.cols;
+        const int64_t n4 = (e1 - e0) >> 2;
+        const float4* src = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(D.w) + e0);
+        for (int64_t i = tid; i < n4; i += kBlockThreads) {
+            const float4 v = src[i];
+            count(v.x); count(v.y); count(v.z); count(v.w);
+        }
+        for (int64_t e = e0 + 4 * n4 + tid; e < e1; e += kBlockThreads)
+            count(reinterpret_cast<const float*>(D.w)[e]);
+    } else {
+        for (int64_t r = r0; r < r1; ++r) {
+            const char* rowp = reinterpret_cast<const char*>(D.w) + r * D.ld * esz;
+            for (int64_t c = tid; c < D.cols; c += kBlockThreads)
+                count(D.dtype == kF32 ? reinterpret_cast<const float*>(rowp)[c]
+                                      : bf16_bits_to_float(reinterpret_cast<const uint16_t*>(rowp)[c]));
+        }
+    }
+    if (PASS == 0) {
+        bad = __syncthreads_or(bad);
+        if (bad && tid == 0 && D.status) atomicOr(reinterpret_cast<unsigned int*>(D.status), kStatusNonfinite);
+    } else {
+        __syncthreads();
+    }
+    for (int i = tid; i < kSelBins; i += kBlockThreads)
+        if (h[i]) atomicAdd(&D.hist[i], h[i]);
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        unsigned int t = atomicAdd(reinterpret_cast<unsigned int*>(&D.state[2]), 1u);
+        s_last = (t == (unsigned int)(D.items - 1));
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+
+    // Last block of this tensor: pick the bucket holding the rem-th largest.
+    const int64_t rem = PASS == 0 ? D.m : (int64_t)__ldcg(&D.state[1]);
+    const int nb = PASS == 2 ? 512 : kSelBins;
+    const int per = nb / kBlockThreads;          // 8 or 2 bins per thread
+    uint32_t sum = 0;
+    for (int i = 0; i < per; ++i) sum += __ldcg(&D.hist[nb - 1 - per * tid - i]);
+    // block-wide inclusive scan of sum (thread order = descending bins)
+    const int warp = tid >> 5, lane = tid & 31;
+    uint32_t incl = sum;
+    for (int off = 1; off < 32; off <<= 1) {
+        uint32_t o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+        if (lane >= off) incl += o;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    uint32_t wbase = 0;
+    for (int w = 0; w < warp; ++w) wbase += s_warp[w];
+    const int64_t excl = (int64_t)wbase + (int64_t)(incl - sum);
+    if (excl < rem && rem <= excl + (int64_t)sum) {
+        int64_t acc = excl;
+        for (int i = 0; i < per; ++i) {
+            const int bin = nb - 1 - per * tid - i;
+            const uint32_t c = __ldcg(&D.hist[bin]);
+            if (acc + c >= rem) {
+                uint32_t np = PASS == 0 ? (uint32_t)bin
+                            : PASS == 1 ? ((prefix << 11) | (uint32_t)bin)
+                                        : ((prefix << 9) | (uint32_t)bin);
+                D.state[0] = np;
+                D.state[1] = (uint32_t)(rem - acc);
+                if (PASS == 2) D.state[3] = np;
+                break;
+            }
+            acc += c;
+        }
+    }
+    __syncthreads();
+    for (int i = tid; i < kSelBins; i += kBlockThreads) D.hist[i] = 0u;
+    if (tid == 0) D.state[2] = 0u;
+}
+
+// ------------------------------------------------------------ elementwise --
+
+// g_w = g_out (copy) or g_w += g_out; dense, n16 16-byte vectors then a tail.
+__global__ void __launch_bounds__(kBlockThreads)
+ste_kernel(const void* __restrict__ g_out, void* __restrict__ g_w, int dtype, int64_t numel,
+           int accumulate, int vec) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int per = dtype == kF32 ? 4 : 8;       // elements per 16 bytes
+    int64_t nvec = vec ? numel / per : 0;
+    const uint4* src = reinterpret_cast<const uint4*>(g_out);
+    uint4* dst = reinterpret_cast<uint4*>(g_w);
+    for (int64_t i = tid; i < nvec; i += stride) {
+        uint4 a = src[i];
+        if (accumulate) {
+            uint4 b = dst[i];
+            if (dtype == kF32) {
+                a.x = __float_as_uint(__fadd_rn(__uint_as_float(b.x), __uint_as_float(a.x)));
+                a.y = __float_as_uint(__fadd_rn(__uint_as_float(b.y), __uint_as_float(a.y)));
+                a.z = __float_as_uint(__fadd_rn(__uint_as_float(b.z), __uint_as_float(a.z)));
+                a.w = __float_as_uint(__fadd_rn(__uint_as_float(b.w), __uint_as_float(a.w)));
+            } else {
+                uint32_t* pa = &a.x;
+                const uint32_t* pb = &b.x;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    float lo = __fadd_rn(bf16_bits_to_float(pb[k] & 0xFFFFu), bf16_bits_to_float(pa[k] & 0xFFFFu));
+                    float hi = __fadd_rn(bf16_bits_to_float(pb[k] >> 16), bf16_bits_to_float(pa[k] >> 16));
+                    pa[k] = (uint32_t)float_to_bf16_bits(lo) | ((uint32_t)float_to_bf16_bits(hi) << 16);
+                }
+            }
+        }
+        dst[i] = a;
+    }
+    for (int64_t e = nvec * per + tid; e < numel; e += stride) {
+        if (dtype == kF32) {
+            float a = reinterpret_cast<const float*>(g_out)[e];
+            float* o = reinterpret_cast<float*>(g_w) + e;
+            *o = accumulate ? __fadd_rn(*o, a) : a;
+        } else {
+            uint16_t a = reinterpret_cast<const uint16_t*>(g_out)[e];
+            uint16_t* o = reinterpret_cast<uint16_t*>(g_w) + e;
+            *o = accumulate ? float_to_bf16_bits(__fadd_rn(bf16_bits_to_float(*o), bf16_bits_to_float(a))) : a;
+        }
+    }
+}
+
+// out[r, c] = (float)q * (float)h[r].  A warp walks a row, one quad (4
+// codes) per lane and step, so the stores are contiguous vectors.  With
+// `words` (int6: cols a multiple of 16 and 4-byte aligned rows; int8: cols a
+// multiple of 4 and aligned rows) lanes read aligned 32-bit words and the
+// 24-bit int6 groups are reassembled with two shuffles; otherwise bytes.
+__global__ void __launch_bounds__(kBlockThreads)
+dequant_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ sf16, int qbits,
+               int per_tensor, int64_t rows, int64_t cols, int64_t prb, void* __restrict__ out,
+               int out_dtype, int vec_out, int words) {
+    const int lane = threadIdx.x & 31;
+    const int sub = lane & 3;
+    const int base = lane & ~3;
+    // int6 group of 4 lanes: lane `sub` needs bytes 3*sub .. 3*sub+2 of the
+    // group's 12, i.e. word a = (3 * sub) / 4 shifted right by 8 * ((3 * sub) % 4)
+    const int a = (3 * sub) >> 2;
+    const int shift = 8 * ((3 * sub) & 3);
+    const int nq = (int)((cols + 3) >> 2);
+    const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += nwarps) {
+        const uint16_t hb = sf16[per_tensor ? 0 : r];
+        const float s = __half2float(*reinterpret_cast<const __half*>(&hb));
+        const uint8_t* prow = packed + r * prb;
+        for (int jb = 0; jb < nq; jb += 32) {
+            const int j = jb + lane;
+            const bool valid = j < nq;
+            const int e0 = 4 * j;
+            int q[4];
+            if (qbits == 6) {
+                uint32_t v;
+                if (words) {
+                    uint32_t word = 0u;
+                    if (valid && sub < 3) word = reinterpret_cast<const uint32_t*>(prow + 3 * (j - sub))[sub];
+                    const uint32_t lo = __shfl_sync(0xFFFFFFFFu, word, base + a);
+                    const uint32_t hi = __shfl_sync(0xFFFFFFFFu, word, base + a + 1);
+                    v = __funnelshift_r(lo, hi, shift);
+                } else {
+                    v = 0u;
+                    if (valid)
+                        v = (uint32_t)prow[3 * j] | ((uint32_t)prow[3 * j + 1] << 8) |
+                            ((uint32_t)prow[3 * j + 2] << 16);
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) q[i] = ((int32_t)(v << (26 - 6 * i))) >> 26;   // sign-extend 6 bits
+            } else {
+                uint32_t v = 0u;
+                if (valid) {
+                    if (words) {
+                        v = *reinterpret_cast<const uint32_t*>(prow + e0);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            if (e0 + i < cols) v |= (uint32_t)prow[e0 + i] << (8 * i);
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) q[i] = ((int32_t)(v << (24 - 8 * i))) >> 24;
+            }
+            if (!valid) continue;
+            float d[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) d[i] = __fmul_rn((float)q[i], s);
+            const bool full = e0 + 3 < cols;
+            if (out_dtype == kF32) {
+                float* o = reinterpret_cast<float*>(out) + r * cols;
+                if (vec_out && full) {
+                    *reinterpret_cast<float4*>(o + e0) = make_float4(d[0], d[1], d[2], d[3]);
+                } else {
+                    for (int i = 0; i < 4; ++i)
+                        if (e0 + i < cols) o[e0 + i] = d[i];
+                }
+            } else {
+                uint16_t* o = reinterpret_cast<uint16_t*>(out) + r * cols;
+                if (vec_out && full) {
+                    *reinterpret_cast<uint2*>(o + e0) =
+                        make_uint2((uint32_t)float_to_bf16_bits(d[0]) | ((uint32_t)float_to_bf16_bits(d[1]) << 16),
+                                   (uint32_t)float_to_bf16_bits(d[2]) | ((uint32_t)float_to_bf16_bits(d[3]) << 16));
+                } else {
+                    for (int i = 0; i < 4; ++i)
+                        if (e0 + i < cols) o[e0 + i] = float_to_bf16_bits(d[i]);
+                }
+            }
+        }
+    }
+}
+
+// Binary16 passthrough of a batch of small tensors: out[r, c] = binary16(w[r, c]).
+struct PassDesc {
+    const void* w;
+    uint16_t* out;
+    int64_t rows, cols, ld;
+    int32_t dtype;
+    int32_t pad;
+};
+
+struct PassParams {
+    int32_t ndesc;
+    int32_t pad;
+    int64_t start[kMaxDesc + 1];   // prefix sums of 1024-element chunks
+    PassDesc d[kMaxDesc];
+};
+
+constexpr int kPassChunk = 1024;
+
+__global__ void __launch_bounds__(kBlockThreads)
+passthrough_kernel(const __grid_constant__ PassParams P) {
+    const int64_t total = P.start[P.ndesc];
+    for (int64_t item = blockIdx.x; item < total; item += gridDim.x) {
+        const int di = find_desc(P.start, P.ndesc, item);
+        const PassDesc& D = P.d[di];
+        const int64_t numel = D.rows * D.cols;
+        const int64_t e_begin = (item - P.start[di]) * kPassChunk;
+        const int64_t e_end = min(numel, e_begin + kPassChunk);
+        for (int64_t e = e_begin + threadIdx.x; e < e_end; e += blockDim.x) {
+            const int64_t r = e / D.cols, c = e - r * D.cols;
+            float x = D.dtype == kF32
+                          ? reinterpret_cast<const float*>(D.w)[r * D.ld + c]
+                          : bf16_bits_to_float(reinterpret_cast<const uint16_t*>(D.w)[r * D.ld + c]);
+            __half h = __float2half_rn(x);
+            D.out[e] = *reinterpret_cast<uint16_t*>(&h);
+        }
+    }
+}
+
+}  // namespace gq

@@ -136,6 +136,18 @@ __device__ __forceinline__ void named_sync(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// max that returns NaN when either input is NaN (the head of a top-m list
+// carries a NaN of its row to the non-finite test).
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+    float r;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+
+__device__ __forceinline__ __nv_bfloat162 as_bf162(uint32_t u) {
+    return *reinterpret_cast<const __nv_bfloat162*>(&u);
+}
+
 // Two floats rounded to bf16 (nearest even), packed low / high.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
@@ -180,8 +192,8 @@ struct Slot {
 
 // The M largest of a multiset of |w| (floats >= +0, compared as floats: the
 // same order as their bit patterns), sorted descending (v[0] largest).
-// fmaxf / fminf ignore NaN; topm_scan reports NaN and +-inf separately by
-// forcing v[0] = +inf, which every later merge carries to the top.
+// The head v[0] is updated with a NaN-propagating max, so a NaN in the row
+// ends up there; +-inf ends up there as the largest |w|.
 template <int M>
 struct TopMF {
     float v[M];
@@ -192,7 +204,7 @@ struct TopMF {
     __device__ __forceinline__ void insert(float x) {
 #pragma unroll
         for (int i = 0; i < M; ++i) {
-            const float hi = fmaxf(v[i], x);
+            const float hi = i == 0 ? fmax_nan(v[i], x) : fmaxf(v[i], x);
             if (i + 1 < M) x = fminf(v[i], x);
             v[i] = hi;
         }
@@ -201,11 +213,11 @@ struct TopMF {
     // max(v0, hi) and max(v1, min(v0, hi), lo) with hi / lo = max / min(a, b)
     __device__ __forceinline__ void insert2(float a, float b) {
         if constexpr (M == 1) {
-            v[0] = fmaxf(v[0], fmaxf(a, b));
+            v[0] = fmax_nan(v[0], fmax_nan(a, b));
         } else if constexpr (M == 2) {
-            const float hi = fmaxf(a, b), lo = fminf(a, b);
+            const float hi = fmax_nan(a, b), lo = fminf(a, b);
             const float t = fminf(v[0], hi);
-            v[0] = fmaxf(v[0], hi);
+            v[0] = fmax_nan(v[0], hi);
             v[1] = fmaxf(v[1], fmaxf(t, lo));
         } else {
             insert(a);
@@ -218,7 +230,7 @@ struct TopMF {
         float r[M];
 #pragma unroll
         for (int i = 0; i < M; ++i) {
-            float x = fmaxf(v[i], b[i]);
+            float x = i == 0 ? fmax_nan(v[0], b[0]) : fmaxf(v[i], b[i]);
 #pragma unroll
             for (int j = 0; j < i; ++j) x = fmaxf(x, fminf(v[j], b[i - 1 - j]));
             r[i] = x;
@@ -244,39 +256,81 @@ struct TopMF {
     }
 };
 
-// Per-thread top-M over the quads j = tl, tl + lpr, ... of a row.  bad
-// accumulates x * 0, which is NaN exactly when some x is NaN or +-inf.
+// Two interleaved top-M lists (M <= 2) of bf16 magnitudes, one per half of
+// a bf16x2 register, on the packed bf16 min / max pipe (two elements per
+// instruction).  bf16 values order exactly like their binary32 widening.
+template <int M>
+struct TopMH {
+    __nv_bfloat162 v[M];
+    __device__ __forceinline__ void init() {
+#pragma unroll
+        for (int i = 0; i < M; ++i) v[i] = as_bf162(0u);
+    }
+    __device__ __forceinline__ void insert2(__nv_bfloat162 a, __nv_bfloat162 b) {
+        if constexpr (M == 1) {
+            v[0] = __hmax2_nan(v[0], __hmax2_nan(a, b));
+        } else {
+            const __nv_bfloat162 hi = __hmax2_nan(a, b), lo = __hmin2(a, b);
+            const __nv_bfloat162 t = __hmin2(v[0], hi);
+            v[0] = __hmax2_nan(v[0], hi);
+            v[1] = __hmax2(v[1], __hmax2(t, lo));
+        }
+    }
+    // the union of both halves as one binary32 list
+    __device__ __forceinline__ void to_f32(TopMF<M>& L) const {
+        float lo[M], hi[M];
+#pragma unroll
+        for (int i = 0; i < M; ++i) {
+            lo[i] = __low2float(v[i]);
+            hi[i] = __high2float(v[i]);
+        }
+#pragma unroll
+        for (int i = 0; i < M; ++i) L.v[i] = lo[i];
+        L.merge(hi);
+    }
+};
+
+// Per-thread top-M over the quads j = tl, tl + lpr, ... of a row.
 template <int DT, int M>
 __device__ __forceinline__ void topm_scan(uint32_t row, int nq, int tl, int lpr, int lg, bool rv, TopMF<M>& L) {
     constexpr uint32_t QB = DT == kF32 ? 16u : 8u;       // bytes of a quad in shared memory
     L.init();
     if (!rv) return;
-    float bad = 0.0f;
     const int nfull = nq >> lg;                           // quads every thread of the slot has
     const uint32_t step = QB * (uint32_t)lpr;
     uint32_t sa = row + QB * (uint32_t)tl;
     int i = 0;
-    for (; i + 2 <= nfull; i += 2, sa += 2 * step) {
-        float a[4], b[4];
-        lds_quad<DT>(sa, 0, a);
-        lds_quad<DT>(sa + step, 0, b);
+    if constexpr (DT == kBF16 && M <= 2) {
+        TopMH<M> H;
+        H.init();
+        for (; i + 2 <= nfull; i += 2, sa += 2 * step) {
+            uint32_t a0, a1, b0, b1;
+            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(a0), "=r"(a1) : "r"(sa));
+            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(b0), "=r"(b1) : "r"(sa + step));
+            H.insert2(as_bf162(a0 & 0x7FFF7FFFu), as_bf162(a1 & 0x7FFF7FFFu));
+            H.insert2(as_bf162(b0 & 0x7FFF7FFFu), as_bf162(b1 & 0x7FFF7FFFu));
+        }
+        for (int j = tl + lpr * i; j < nq; j += lpr, sa += step) {
+            uint32_t a0, a1;
+            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(a0), "=r"(a1) : "r"(sa));
+            H.insert2(as_bf162(a0 & 0x7FFF7FFFu), as_bf162(a1 & 0x7FFF7FFFu));
+        }
+        H.to_f32(L);
+    } else {
+        for (; i + 2 <= nfull; i += 2, sa += 2 * step) {
+            float a[4], b[4];
+            lds_quad<DT>(sa, 0, a);
+            lds_quad<DT>(sa + step, 0, b);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            L.insert2(fabsf(a[k]), fabsf(b[k]));
-            bad = __fmaf_rn(a[k], 0.0f, bad);
-            bad = __fmaf_rn(b[k], 0.0f, bad);
+            for (int k = 0; k < 4; ++k) L.insert2(fabsf(a[k]), fabsf(b[k]));
+        }
+        for (int j = tl + lpr * i; j < nq; j += lpr, sa += step) {
+            float a[4];
+            lds_quad<DT>(sa, 0, a);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) L.insert(fabsf(a[k]));
         }
     }
-    for (int j = tl + lpr * i; j < nq; j += lpr, sa += step) {
-        float a[4];
-        lds_quad<DT>(sa, 0, a);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            L.insert(fabsf(a[k]));
-            bad = __fmaf_rn(a[k], 0.0f, bad);
-        }
-    }
-    if (bad != bad) L.v[0] = __int_as_float(0x7F800000);   // +inf marks a non-finite row
 }
 
 // MSB-first radix select (8+8+8+7 bits) over the shared-memory row, for a
@@ -429,6 +483,41 @@ __device__ __forceinline__ void round8(const float x[8], const Scale& S, float n
     }
 }
 
+// Rounded quotients of two quads for the branch-free loop: n[k] (integer-
+// valued floats) and b[k] = kMagic + n[k] (the code bits), with one warp
+// vote for both rare events: a quotient within 2^-13 of a half-integer
+// (exact division for that lane) and, with CLAMP, a code beyond qmax.
+template <bool CLAMP>
+__device__ __forceinline__ void round8_fast(const float x[8], float rcp, float s, float qmaxf, float n[8],
+                                            float b[8]) {
+    float y[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        y[k] = __fmul_rn(x[k], rcp);
+        b[k] = __fadd_rn(y[k], kMagic);
+        n[k] = __fsub_rn(b[k], kMagic);
+    }
+    float dmax = fabsf(__fsub_rn(y[0], n[0]));
+#pragma unroll
+    for (int k = 1; k < 8; ++k) dmax = fmaxf(dmax, fabsf(__fsub_rn(y[k], n[k])));
+    const bool near = dmax > kNearHalf;
+    bool rare = near;
+    if (CLAMP) {
+        float nmax = fabsf(n[0]);
+#pragma unroll
+        for (int k = 1; k < 8; ++k) nmax = fmaxf(nmax, fabsf(n[k]));
+        rare |= nmax > qmaxf;
+    }
+    if (__any_sync(0xFFFFFFFFu, rare)) {
+        if (near) exact_round8(x, s, n);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            if (CLAMP) n[k] = fminf(fmaxf(n[k], -qmaxf), qmaxf);
+            b[k] = __fadd_rn(n[k], kMagic);
+        }
+    }
+}
+
 // Stores of one quad for a compile-time output configuration, at running
 // pointers: pd (w_hat quad), pc (4 code bytes), pp (int8: 4 bytes; int6: this
 // lane's 32-bit word of its 4-lane group, unused by the group's 4th lane).
@@ -500,24 +589,9 @@ __device__ __forceinline__ void quantize_row_fast(uint32_t row, int nq, int tl, 
         float x[8];
         lds_quad<DT>(sa, 0, x);
         lds_quad<DT>(sa + step, 0, x + 4);
-        float n[8];
-        round8<false>(x, S, n);
+        // only codes of |w| > c can exceed qmax, so the clamp is a rare path
         float q[8], b[8];
-        if (CLAMP) {
-            // only codes of |w| > c can exceed qmax: clamp when the warp has one
-            float nmax = fabsf(n[0]);
-#pragma unroll
-            for (int k = 1; k < 8; ++k) nmax = fmaxf(nmax, fabsf(n[k]));
-            if (__any_sync(0xFFFFFFFFu, nmax > qmaxf)) {
-#pragma unroll
-                for (int k = 0; k < 8; ++k) n[k] = fminf(fmaxf(n[k], -qmaxf), qmaxf);
-            }
-        }
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            q[k] = n[k];
-            b[k] = __fadd_rn(q[k], kMagic);
-        }
+        round8_fast<CLAMP>(x, rcp, s, qmaxf, q, b);
         put_quad<DT, OUT>(pd, pc, pp, rv, sub, q, b, s);
         put_quad<DT, OUT>(pd + sd, pc + sc, pp + sp, rv, sub, q + 4, b + 4, s);
         sa += 2 * step;
@@ -530,14 +604,8 @@ __device__ __forceinline__ void quantize_row_fast(uint32_t row, int nq, int tl, 
         const bool valid = rv && (tl + lpr * i < nq);
         float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         if (valid) lds_quad<DT>(sa, 0, x);
-        float n[8];
-        round8<false>(x, S, n);
-        float q[4], b[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            q[k] = CLAMP ? fminf(fmaxf(n[k], -qmaxf), qmaxf) : n[k];
-            b[k] = __fadd_rn(q[k], kMagic);
-        }
+        float q[8], b[8];
+        round8_fast<CLAMP>(x, rcp, s, qmaxf, q, b);
         put_quad<DT, OUT>(pd, pc, pp, valid, sub, q, b, s);
         sa += step;
         pd += sd;
