@@ -219,14 +219,18 @@ gq_status run_rows_tma(std::vector<RowDesc>& rows, cudaStream_t stream) {
     for (const RowDesc& D : rows) max_row = std::max<int64_t>(max_row, D.cols * (D.dtype == kF32 ? 4 : 2));
     const int sb = max_row <= kTmaStageBytes ? kTmaStageBytes : (int)((max_row + 15) / 16 * 16);
     const int nstages = max_row <= kTmaStageBytes ? 3 : 2;
+    // two tile-teams of 8 warps take alternate tiles when a third stage is
+    // left for prefetching; a row then needs half as many threads
+    const int teams = nstages == 3 ? 2 : 1;
+    const int team_threads = kTmaConsumers / teams;
     for (RowDesc& D : rows) {
         const int64_t row_bytes = D.cols * (D.dtype == kF32 ? 4 : 2);
         const int64_t rmax = sb / row_bytes;
         // radix selection (m > 8, per row) runs on whole warps
         const bool whole_warps = !D.clip_in && D.m > kTopMax;
         int lpr = 8;
-        while (lpr < kTmaConsumers && (kTmaConsumers / lpr > rmax || (whole_warps && lpr < 32))) lpr *= 2;
-        const int64_t slots = kTmaConsumers / lpr;
+        while (lpr < team_threads && (team_threads / lpr > rmax || (whole_warps && lpr < 32))) lpr *= 2;
+        const int64_t slots = team_threads / lpr;
         D.tile_rows = (int32_t)(rmax / slots * slots);
         D.lanes_per_row = lpr;
         D.out_mode = tma_out_mode(D);
@@ -248,6 +252,7 @@ gq_status run_rows_tma(std::vector<RowDesc>& rows, cudaStream_t stream) {
         P.ndesc = nd;
         P.nstages = nstages;
         P.stage_bytes = sb;
+        P.teams = teams;
         int64_t acc = 0;
         for (int i = 0; i < nd; ++i) {
             P.start[i] = acc;

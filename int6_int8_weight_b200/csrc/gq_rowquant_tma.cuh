@@ -48,7 +48,8 @@ struct TmaParams {
     int32_t ndesc;
     int32_t nstages;
     int32_t stage_bytes;
-    int32_t pad;
+    int32_t teams;       // tile-teams: the consumer warps split into `teams` groups
+                         // that take alternate tiles (1 or 2)
     int64_t start[kMaxDesc + 1];   // prefix sums of tiles
     RowDesc d[kMaxDesc];
 };
@@ -56,7 +57,7 @@ struct TmaParams {
 // Shared memory after the stages: mbarriers, per-warp selection lists,
 // per-slot broadcast records and per-slot radix histograms.
 constexpr int kBcastWords = 8;
-constexpr int kTmaExtraBytes = 2 * kTmaMaxStages * 8 + 2 * kTmaConsumerWarps * kTopMax * 4 +
+constexpr int kTmaExtraBytes = 3 * kTmaMaxStages * 8 + 2 * kTmaConsumerWarps * kTopMax * 4 +
                                kTmaConsumerWarps * kBcastWords * 4 + kTmaConsumerWarps * 256 * 4;
 
 // ------------------------------------------------------------- PTX glue --
@@ -874,8 +875,15 @@ rowquant_tma_kernel(const __grid_constant__ TmaParams P) {
     const int S = P.nstages;
     const uint32_t SB = (uint32_t)P.stage_bytes;
     unsigned char* extra = smem + (size_t)S * SB;
+    // Two "full" barriers per stage, used on alternate fills: fill k of stage
+    // s completes phase k / 2 of full[2 s + k % 2].  A tile-team lags at most
+    // one fill of a stage behind (the other team's tile), and a one-bit
+    // parity wait stays unambiguous only while the waiter is less than two
+    // phases of its barrier behind, which alternation guarantees.
     uint64_t* full = reinterpret_cast<uint64_t*>(extra);
-    uint64_t* empty = full + kTmaMaxStages;
+    uint64_t* empty = full + 2 * kTmaMaxStages;
+    auto full_bar = [&](int stage, int fill) { return smem_u32(&full[2 * stage + (fill & 1)]); };
+    auto full_parity = [](int fill) { return (uint32_t)((fill >> 1) & 1); };
     float* lists = reinterpret_cast<float*>(empty + kTmaMaxStages);                        // [2][warp][kTopMax]
     uint32_t* bcast = reinterpret_cast<uint32_t*>(lists + 2 * kTmaConsumerWarps * kTopMax);  // [slot][8]
     uint32_t* hist = bcast + kTmaConsumerWarps * kBcastWords;                          // [slot][256]
@@ -883,8 +891,9 @@ rowquant_tma_kernel(const __grid_constant__ TmaParams P) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(smem_u32(&full[s]), 1);
-            mbar_init(smem_u32(&empty[s]), kTmaConsumerWarps);
+            mbar_init(smem_u32(&full[2 * s]), 1);
+            mbar_init(smem_u32(&full[2 * s + 1]), 1);
+            mbar_init(smem_u32(&empty[s]), kTmaConsumerWarps / P.teams);
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -913,44 +922,53 @@ rowquant_tma_kernel(const __grid_constant__ TmaParams P) {
             const int64_t nr = min((int64_t)D.tile_rows, D.rows - r0);
             const int esz = D.dtype == kF32 ? 4 : 2;
             const uint32_t row_bytes = (uint32_t)(D.cols * esz);
-            const uint32_t full_bar = smem_u32(&full[s]);
+            const uint32_t fb = full_bar(s, k);
             const uint32_t dst = smem_base + (uint32_t)s * SB;
             const char* src = reinterpret_cast<const char*>(D.w) + r0 * D.ld * esz;
-            mbar_arrive_expect_tx(full_bar, (uint32_t)nr * row_bytes);
+            mbar_arrive_expect_tx(fb, (uint32_t)nr * row_bytes);
             if (D.ld == D.cols) {
-                bulk_g2s(dst, src, (uint32_t)nr * row_bytes, full_bar);
+                bulk_g2s(dst, src, (uint32_t)nr * row_bytes, fb);
             } else {
                 for (int64_t i = 0; i < nr; ++i)
-                    bulk_g2s(dst + (uint32_t)i * row_bytes, src + i * D.ld * esz, row_bytes, full_bar);
+                    bulk_g2s(dst + (uint32_t)i * row_bytes, src + i * D.ld * esz, row_bytes, fb);
             }
         }
         if (!ok) {
             // wait (bounded) for the copies already issued before leaving
             for (int i = max(0, it - S); i < it; ++i)
-                (void)mbar_wait(smem_u32(&full[i % S]), (uint32_t)((i / S) & 1));
+                (void)mbar_wait(full_bar(i % S, i / S), full_parity(i / S));
         }
         return;
     }
 
     // -------------------------------------------------------- consumers --
+    // Tile-team `team` takes the tiles it == team (mod teams); its slots are
+    // numbered globally (slot = consumer thread / lpr), so the shared records
+    // of different tile-teams never overlap.
+    const int teams = P.teams;
+    const int wpt = kTmaConsumerWarps / teams;       // warps per tile-team
+    const int team = warp / wpt;
+    const int team_threads = wpt * 32;
     int it = 0;
     int prev_lpr = 0;
-    int seq = 0;          // rows this warp's team has processed since the last shape change
+    int seq = 0;          // rows this warp's slot has processed since the last shape change
     for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
+        if (it % teams != team) continue;
         const int s = it % S;
         const int k = it / S;
         const int di = find_desc(P.start, P.ndesc, t);
         const RowDesc& D = P.d[di];
         const int lpr = D.lanes_per_row;
         if (lpr != prev_lpr) {
-            // the slot shape changes: no warp may still use the old slots'
-            // shared records (every consumer warp takes this branch on the
-            // same tile)
-            if (prev_lpr != 0) named_sync(0, kTmaConsumers);
+            // the slot shape changes: no warp of this tile-team may still use
+            // the old slots' shared records (all its warps take this branch on
+            // the same tile); team 0 meets at barrier 0, team 1 at barrier 15
+            // (free: a 16-warp row needs a single tile-team)
+            if (prev_lpr != 0) named_sync(team == 0 ? 0 : 15, team_threads);
             prev_lpr = lpr;
             seq = 0;
         }
-        if (!mbar_wait(smem_u32(&full[s]), (uint32_t)(k & 1))) {
+        if (!mbar_wait(full_bar(s, k), full_parity(k))) {
             if (lane == 0 && D.status) atomicOr(reinterpret_cast<unsigned int*>(D.status), kStatusTimeout);
             break;
         }
@@ -960,18 +978,19 @@ rowquant_tma_kernel(const __grid_constant__ TmaParams P) {
         const uint32_t stage = smem_base + (uint32_t)s * SB;
         Slot T;
         T.init(lpr, warp, lane);
-        const int slots = kTmaConsumers >> T.lg;
+        const int slots = team_threads >> T.lg;          // slots of this tile-team
+        const int lslot = T.slot - team * slots;         // slot index within it
         if (lpr < 32) {
             const int rounds = (nr + slots - 1) / slots;
             for (int rd = 0; rd < rounds; ++rd) {
-                const int i = rd * slots + T.slot;
+                const int i = rd * slots + lslot;
                 const bool rv = i < nr;
                 const uint32_t row = stage + (uint32_t)(rv ? i : 0) * row_bytes;
                 if (D.dtype == kF32) process_row_sub<kF32>(D, r0 + i, row, T, rv);
                 else process_row_sub<kBF16>(D, r0 + i, row, T, rv);
             }
         } else {
-            for (int i = T.slot; i < nr; i += slots, ++seq) {
+            for (int i = lslot; i < nr; i += slots, ++seq) {
                 const uint32_t row = stage + (uint32_t)i * row_bytes;
                 uint32_t* bc = bcast + T.slot * kBcastWords;
                 uint32_t* hs = hist + T.slot * 256;

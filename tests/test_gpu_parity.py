@@ -455,3 +455,29 @@ def test_pipelined_strided_bf16_and_two_stage_rows(gq):
     run_export_and_check(gq, w, 6, 0.9999, what="two-stage 20000 cols")
     run_train_and_check(gq, w, 8, 0.3, what="two-stage 20000 cols radix")
     run_export_and_check(gq, w, 6, 0.999, per_tensor=True, what="two-stage per-tensor")
+
+
+def test_pipelined_repeatability_stress(gq):
+    """Many back-to-back launches over many tiles per block (both tile-teams
+    busy, every stage reused many times): outputs must be identical launch
+    after launch and match the oracle on sampled rows; status stays 0."""
+    rng = np.random.default_rng(13)
+    for (rows, cols, dt) in ((65536, 512, torch.bfloat16), (16384, 2048, torch.float32),
+                             (2048, 16384, torch.float32)):
+        W = synth.draw_bandwidth_matrix(rows, cols, 7, device=DEV).to(dt)
+        first = None
+        for it in range(12):
+            (o,) = gq.export_pack([gq.Request(W, 6, 0.9999, want_dq=True)])
+            assert o.status == 0
+            if first is None:
+                first = o
+                idx = np.unique(np.concatenate([[0, rows - 1], rng.integers(0, rows, 24)]))
+                ti = torch.from_numpy(idx).to(DEV)
+                ref = oracle.quantize(to_host(W.index_select(0, ti)), 6, 0.9999, export=True)
+                assert_same(to_host(o.packed.index_select(0, ti)), ref.packed, f"{rows}x{cols} packed")
+                assert_same(to_host(o.dq.index_select(0, ti)), ref.dq, f"{rows}x{cols} dq")
+            else:
+                assert torch.equal(o.packed, first.packed), (rows, cols, it)
+                assert torch.equal(o.dq.view(torch.int16 if dt == torch.bfloat16 else torch.int32),
+                                   first.dq.view(torch.int16 if dt == torch.bfloat16 else torch.int32)), (rows, cols, it)
+                assert torch.equal(o.scale_f16.view(torch.int16), first.scale_f16.view(torch.int16))
