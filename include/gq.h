@@ -58,7 +58,12 @@
  *  - Outputs are dense row-major [rows, cols] (packed: [rows, packed row
  *    bytes]); the input may be strided (ld >= cols elements).
  *  - A tensor with rows == 0 or cols == 0 is a no-op; its pointers may be NULL.
- *  - No call synchronizes, spins, traps or asserts on the device.
+ *  - No call synchronizes with the host, traps or asserts on the device.  The
+ *    only waits on the device are the fused row kernel's waits for its own
+ *    bulk copies into shared memory (and its consumers' waits for one
+ *    another); each gives up after about 4 s of %globaltimer, drains the
+ *    copies still in flight (again bounded), sets GQ_STATUS_TIMEOUT in the
+ *    descriptor's status word and lets the launch end.
  */
 #ifndef GQ_H
 #define GQ_H
@@ -89,7 +94,7 @@ typedef enum gq_status {
     GQ_ERR_RANGE = 5,         /* reserved (device-side: GQ_STATUS_RANGE) */
     GQ_ERR_NONFINITE = 6,     /* reserved (device-side: GQ_STATUS_NONFINITE) */
     GQ_ERR_CUDA = 7,          /* a CUDA runtime call or launch failed */
-    GQ_ERR_TIMEOUT = 8        /* reserved: no call waits on the device */
+    GQ_ERR_TIMEOUT = 8        /* reserved (device-side: GQ_STATUS_TIMEOUT) */
 } gq_status;
 
 typedef enum gq_dtype { GQ_F32 = 0, GQ_BF16 = 1 } gq_dtype;
@@ -102,6 +107,7 @@ typedef enum gq_scale_mode {
 /* Bits OR-ed into d_status[i]. */
 #define GQ_STATUS_NONFINITE 0x1  /* a NaN or +-inf in the tensor */
 #define GQ_STATUS_RANGE     0x2  /* binary16(c / qmax) overflowed to inf */
+#define GQ_STATUS_TIMEOUT   0x4  /* a bounded wait on the device gave up */
 
 /* Kinds returned by gq_plan_kind. */
 #define GQ_KIND_RAW  0  /* not floating point: stored as is */
