@@ -4,7 +4,8 @@
 // Arithmetic contract (the definitions in include/gq.h): every floating-point
 // step that decides an output bit is one correctly rounded binary32 operation,
 // written with the explicit-rounding intrinsics (__fmul_rn, __fadd_rn,
-// __fdiv_rn, __frcp_rn) so the compiler cannot contract or reassociate it.
+// __fdiv_rn, __frcp_rn) or the paired .rn f32x2 instructions (two independent
+// binary32 lanes), so the compiler cannot contract or reassociate it.
 #pragma once
 
 #include <cuda_bf16.h>

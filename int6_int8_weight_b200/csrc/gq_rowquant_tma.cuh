@@ -34,7 +34,7 @@ namespace gq {
 
 constexpr int kTmaConsumerWarps = 16;
 constexpr int kTmaConsumers = kTmaConsumerWarps * 32;
-constexpr int kTmaThreads = kTmaConsumers + 32;
+constexpr int kTmaThreads = kTmaConsumers;   // no producer warp: consumers refill the stages
 constexpr int kTmaMaxStages = 4;
 constexpr uint32_t kStatusTimeout = 0x4u;
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;   // 4 s
@@ -54,8 +54,8 @@ struct TmaParams {
     RowDesc d[kMaxDesc];
 };
 
-// Shared memory after the stages: mbarriers, per-warp selection lists,
-// per-slot broadcast records and per-slot radix histograms.
+// Shared memory after the stages: mbarriers and stage counters, per-warp
+// selection lists, per-slot broadcast records and per-slot radix histograms.
 constexpr int kBcastWords = 8;
 constexpr int kTmaExtraBytes = 3 * kTmaMaxStages * 8 + 2 * kTmaConsumerWarps * kTopMax * 4 +
                                kTmaConsumerWarps * kBcastWords * 4 + kTmaConsumerWarps * 256 * 4;
@@ -95,6 +95,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "r"(bar), "r"(parity)
         : "memory");
     return done != 0;
+}
+
+// Shared-memory fetch-and-add with acquire-release ordering at CTA scope.
+__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t addr, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(addr), "r"(v) : "memory");
+    return old;
 }
 
 // Bounded wait for the completion of the phase with the given parity.
@@ -153,6 +160,32 @@ __device__ __forceinline__ __nv_bfloat162 as_bf162(uint32_t u) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Two binary32 lanes in one 64-bit register for the paired f32x2 operations
+// (each lane one correctly rounded binary32 operation).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
 }
 
 // ------------------------------------------------------------------ slot --
@@ -447,9 +480,8 @@ __device__ __forceinline__ void write_row_scalars(const RowDesc& D, int64_t r, c
 
 // ------------------------------------------------------ element kernel --
 
-// Exact quotients for the lanes where the guard fired (rare); arguments and
-// results travel in registers.
-__device__ __noinline__ float4 exact_round4(float a, float b, float c, float d, float s) {
+// Exact quotients for the lanes where the guard fired (rare).
+__device__ __forceinline__ float4 exact_round4(float a, float b, float c, float d, float s) {
     return make_float4(__fsub_rn(__fadd_rn(__fdiv_rn(a, s), kMagic), kMagic),
                        __fsub_rn(__fadd_rn(__fdiv_rn(b, s), kMagic), kMagic),
                        __fsub_rn(__fadd_rn(__fdiv_rn(c, s), kMagic), kMagic),
@@ -487,20 +519,26 @@ __device__ __forceinline__ void round8(const float x[8], const Scale& S, float n
 // Rounded quotients of two quads for the branch-free loop: n[k] (integer-
 // valued floats) and b[k] = kMagic + n[k] (the code bits), with one warp
 // vote for both rare events: a quotient within 2^-13 of a half-integer
-// (exact division for that lane) and, with CLAMP, a code beyond qmax.
+// (exact division for that lane) and, with CLAMP, a code beyond qmax.  The
+// products and sums run on element pairs (f32x2), each lane of which is the
+// same correctly rounded binary32 operation as the scalar form.
 template <bool CLAMP>
 __device__ __forceinline__ void round8_fast(const float x[8], float rcp, float s, float qmaxf, float n[8],
                                             float b[8]) {
-    float y[8];
+    float e[8];
+    const uint64_t R2 = f2_pack(rcp, rcp), M2 = f2_pack(kMagic, kMagic);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        y[k] = __fmul_rn(x[k], rcp);
-        b[k] = __fadd_rn(y[k], kMagic);
-        n[k] = __fsub_rn(b[k], kMagic);
+    for (int k = 0; k < 8; k += 2) {
+        const uint64_t Y = f2_mul(f2_pack(x[k], x[k + 1]), R2);
+        const uint64_t B = f2_add(Y, M2);
+        const uint64_t N = f2_sub(B, M2);
+        f2_unpack(f2_sub(Y, N), e[k], e[k + 1]);
+        f2_unpack(B, b[k], b[k + 1]);
+        f2_unpack(N, n[k], n[k + 1]);
     }
-    float dmax = fabsf(__fsub_rn(y[0], n[0]));
+    float dmax = fabsf(e[0]);
 #pragma unroll
-    for (int k = 1; k < 8; ++k) dmax = fmaxf(dmax, fabsf(__fsub_rn(y[k], n[k])));
+    for (int k = 1; k < 8; ++k) dmax = fmaxf(dmax, fabsf(e[k]));
     const bool near = dmax > kNearHalf;
     bool rare = near;
     if (CLAMP) {
@@ -519,6 +557,10 @@ __device__ __forceinline__ void round8_fast(const float x[8], float rcp, float s
     }
 }
 
+// (0x4B400000 - 32) * (1 + 64 + 4096 + 262144) mod 2^32: the offset that
+// turns the sum of four code words b into the biased 24-bit group.
+constexpr uint32_t kSixBias = 0x1ABDF7E0u;
+
 // Stores of one quad for a compile-time output configuration, at running
 // pointers: pd (w_hat quad), pc (4 code bytes), pp (int8: 4 bytes; int6: this
 // lane's 32-bit word of its 4-lane group, unused by the group's 4th lane).
@@ -530,12 +572,14 @@ __device__ __forceinline__ void put_quad(char* pd, int8_t* pc, uint8_t* pp, bool
     const uint32_t b0 = __float_as_uint(b[0]), b1 = __float_as_uint(b[1]);
     const uint32_t b2 = __float_as_uint(b[2]), b3 = __float_as_uint(b[3]);
     if constexpr ((OUT & kOutDq) != 0) {
+        float w[4];
+        const uint64_t S2 = f2_pack(s, s);
+        f2_unpack(f2_mul(f2_pack(q[0], q[1]), S2), w[0], w[1]);
+        f2_unpack(f2_mul(f2_pack(q[2], q[3]), S2), w[2], w[3]);
         if constexpr (DT == kF32) {
-            const float4 d = make_float4(__fmul_rn(q[0], s), __fmul_rn(q[1], s), __fmul_rn(q[2], s), __fmul_rn(q[3], s));
-            if (valid) *reinterpret_cast<float4*>(pd) = d;
+            if (valid) *reinterpret_cast<float4*>(pd) = make_float4(w[0], w[1], w[2], w[3]);
         } else {
-            const uint2 d = make_uint2(pack_bf16x2(__fmul_rn(q[0], s), __fmul_rn(q[1], s)),
-                                       pack_bf16x2(__fmul_rn(q[2], s), __fmul_rn(q[3], s)));
+            const uint2 d = make_uint2(pack_bf16x2(w[0], w[1]), pack_bf16x2(w[2], w[3]));
             if (valid) *reinterpret_cast<uint2*>(pd) = d;
         }
     }
@@ -549,10 +593,16 @@ __device__ __forceinline__ void put_quad(char* pd, int8_t* pc, uint8_t* pp, bool
         }
     }
     if constexpr ((OUT & kOutPacked) != 0 && (OUT & kOutSix) != 0) {
-        // four lanes pack 16 codes into three aligned 32-bit words
-        const uint32_t v24 = (b0 & 0x3Fu) | ((b1 << 6) & 0xFC0u) | ((b2 << 12) & 0x3F000u) | ((b3 << 18) & 0xFC0000u);
+        // The 24-bit group of the quad without per-field masks: u = q + 32 is
+        // in [1, 63], so U = u0 + 64 u1 + 4096 u2 + 262144 u3 has no carries
+        // between fields, and a code's two's-complement field is u ^ 32.  As
+        // integers b = 0x4B400000 + q, so U = b0 + 64 b1 + 4096 b2 + 262144 b3
+        // - kSixBias (mod 2^32).
+        const uint32_t v24 = ((b0 + 64u * b1 + 4096u * b2 + 262144u * b3) - kSixBias) ^ 0x820820u;
+        // four lanes pack 16 codes into three aligned 32-bit words: word sub
+        // is bytes 3 sub .. 3 sub + 3 of the group pair (this lane, next lane)
         const uint32_t nxt = __shfl_down_sync(0xFFFFFFFFu, v24, 1);
-        const uint32_t word = (v24 >> (8 * sub)) | (nxt << (24 - 8 * sub));
+        const uint32_t word = __byte_perm(v24, nxt, (uint32_t)(0x654254214210ull >> (16 * sub)) & 0xFFFFu);
         if (valid && sub < 3) *reinterpret_cast<uint32_t*>(pp) = word;
     }
 }
@@ -869,6 +919,28 @@ __device__ __forceinline__ void process_row_team(const RowDesc& D, int64_t r, ui
 
 // ------------------------------------------------------------- kernel --
 
+// Start the bulk copy of this CTA's tile number `it` (global tile
+// blockIdx.x + it * gridDim.x) into stage it % S as fill it / S of that
+// stage.  `di` is the caller's descriptor cursor: tiles it issues only grow.
+__device__ __forceinline__ void issue_tile(const TmaParams& P, int it, int& di, uint32_t smem_base, uint32_t SB,
+                                           int S, uint32_t bar) {
+    const int64_t t = blockIdx.x + (int64_t)it * gridDim.x;
+    while (t >= P.start[di + 1]) ++di;
+    const RowDesc& D = P.d[di];
+    const int64_t r0 = (t - P.start[di]) * D.tile_rows;
+    const int64_t nr = min((int64_t)D.tile_rows, D.rows - r0);
+    const int esz = D.dtype == kF32 ? 4 : 2;
+    const uint32_t row_bytes = (uint32_t)(D.cols * esz);
+    const uint32_t dst = smem_base + (uint32_t)(it % S) * SB;
+    const char* src = reinterpret_cast<const char*>(D.w) + r0 * D.ld * esz;
+    mbar_arrive_expect_tx(bar, (uint32_t)nr * row_bytes);
+    if (D.ld == D.cols) {
+        bulk_g2s(dst, src, (uint32_t)nr * row_bytes, bar);
+    } else {
+        for (int64_t i = 0; i < nr; ++i) bulk_g2s(dst + (uint32_t)i * row_bytes, src + i * D.ld * esz, row_bytes, bar);
+    }
+}
+
 __global__ void __launch_bounds__(kTmaThreads, 1)
 rowquant_tma_kernel(const __grid_constant__ TmaParams P) {
     extern __shared__ __align__(128) unsigned char smem[];
@@ -881,82 +953,51 @@ rowquant_tma_kernel(const __grid_constant__ TmaParams P) {
     // parity wait stays unambiguous only while the waiter is less than two
     // phases of its barrier behind, which alternation guarantees.
     uint64_t* full = reinterpret_cast<uint64_t*>(extra);
-    uint64_t* empty = full + 2 * kTmaMaxStages;
+    // done[s]: warps that have finished with stage s, over all its fills.
+    // Every fill is read by one tile-team of wpt warps, so the warp whose
+    // increment makes the count a multiple of wpt is the last reader of the
+    // fill and starts the next one.
+    uint32_t* done = reinterpret_cast<uint32_t*>(full + 2 * kTmaMaxStages);
     auto full_bar = [&](int stage, int fill) { return smem_u32(&full[2 * stage + (fill & 1)]); };
     auto full_parity = [](int fill) { return (uint32_t)((fill >> 1) & 1); };
-    float* lists = reinterpret_cast<float*>(empty + kTmaMaxStages);                        // [2][warp][kTopMax]
+    float* lists = reinterpret_cast<float*>(full + 3 * kTmaMaxStages);                     // [2][warp][kTopMax]
     uint32_t* bcast = reinterpret_cast<uint32_t*>(lists + 2 * kTmaConsumerWarps * kTopMax);  // [slot][8]
     uint32_t* hist = bcast + kTmaConsumerWarps * kBcastWords;                          // [slot][256]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t ntiles = P.start[P.ndesc];
+    const uint32_t smem_base = smem_u32(smem);
+    int di_issue = 0;     // descriptor cursor of the tiles this thread issues
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(smem_u32(&full[2 * s]), 1);
             mbar_init(smem_u32(&full[2 * s + 1]), 1);
-            mbar_init(smem_u32(&empty[s]), kTmaConsumerWarps / P.teams);
+            done[s] = 0u;
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        // first fill of every stage
+        for (int it = 0; it < S && blockIdx.x + (int64_t)it * gridDim.x < ntiles; ++it)
+            issue_tile(P, it, di_issue, smem_base, SB, S, full_bar(it, 0));
     }
     __syncthreads();
 
-    const int64_t ntiles = P.start[P.ndesc];
-    const uint32_t smem_base = smem_u32(smem);
-
-    if (warp == kTmaConsumerWarps) {
-        // ---------------------------------------------------- producer --
-        if (lane != 0) return;
-        int it = 0;
-        bool ok = true;
-        for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
-            const int s = it % S;
-            const int k = it / S;
-            const int di = find_desc(P.start, P.ndesc, t);
-            const RowDesc& D = P.d[di];
-            if (k > 0 && !mbar_wait(smem_u32(&empty[s]), (uint32_t)((k - 1) & 1))) {
-                if (D.status) atomicOr(reinterpret_cast<unsigned int*>(D.status), kStatusTimeout);
-                ok = false;
-                break;
-            }
-            const int64_t r0 = (t - P.start[di]) * D.tile_rows;
-            const int64_t nr = min((int64_t)D.tile_rows, D.rows - r0);
-            const int esz = D.dtype == kF32 ? 4 : 2;
-            const uint32_t row_bytes = (uint32_t)(D.cols * esz);
-            const uint32_t fb = full_bar(s, k);
-            const uint32_t dst = smem_base + (uint32_t)s * SB;
-            const char* src = reinterpret_cast<const char*>(D.w) + r0 * D.ld * esz;
-            mbar_arrive_expect_tx(fb, (uint32_t)nr * row_bytes);
-            if (D.ld == D.cols) {
-                bulk_g2s(dst, src, (uint32_t)nr * row_bytes, fb);
-            } else {
-                for (int64_t i = 0; i < nr; ++i)
-                    bulk_g2s(dst + (uint32_t)i * row_bytes, src + i * D.ld * esz, row_bytes, fb);
-            }
-        }
-        if (!ok) {
-            // wait (bounded) for the copies already issued before leaving
-            for (int i = max(0, it - S); i < it; ++i)
-                (void)mbar_wait(full_bar(i % S, i / S), full_parity(i / S));
-        }
-        return;
-    }
-
-    // -------------------------------------------------------- consumers --
     // Tile-team `team` takes the tiles it == team (mod teams); its slots are
-    // numbered globally (slot = consumer thread / lpr), so the shared records
-    // of different tile-teams never overlap.
+    // numbered globally (slot = thread / lpr), so the shared records of
+    // different tile-teams never overlap.
     const int teams = P.teams;
     const int wpt = kTmaConsumerWarps / teams;       // warps per tile-team
     const int team = warp / wpt;
     const int team_threads = wpt * 32;
     int it = 0;
+    int di = 0;           // tiles come in increasing order: their descriptors too
     int prev_lpr = 0;
     int seq = 0;          // rows this warp's slot has processed since the last shape change
     for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
         if (it % teams != team) continue;
         const int s = it % S;
         const int k = it / S;
-        const int di = find_desc(P.start, P.ndesc, t);
+        while (t >= P.start[di + 1]) ++di;
         const RowDesc& D = P.d[di];
         const int lpr = D.lanes_per_row;
         if (lpr != prev_lpr) {
@@ -969,7 +1010,11 @@ rowquant_tma_kernel(const __grid_constant__ TmaParams P) {
             seq = 0;
         }
         if (!mbar_wait(full_bar(s, k), full_parity(k))) {
-            if (lane == 0 && D.status) atomicOr(reinterpret_cast<unsigned int*>(D.status), kStatusTimeout);
+            if (lane == 0) {
+                if (D.status) atomicOr(reinterpret_cast<unsigned int*>(D.status), kStatusTimeout);
+                // wait (bounded) for the copies that may still be in flight
+                for (int j = it; j < it + S; ++j) (void)mbar_wait(full_bar(j % S, j / S), full_parity(j / S));
+            }
             break;
         }
         const int64_t r0 = (t - P.start[di]) * D.tile_rows;
@@ -998,8 +1043,14 @@ rowquant_tma_kernel(const __grid_constant__ TmaParams P) {
                 else process_row_team<kBF16>(D, r0 + i, row, T, lists, bc, hs, seq);
             }
         }
+        // Release the stage: the acquire-release increment orders this warp's
+        // reads of the stage before the refill that the last reader starts.
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
+        if (lane == 0) {
+            const uint32_t before = atom_add_acq_rel(smem_u32(&done[s]), 1u);
+            if ((before + 1u) % (uint32_t)wpt == 0u && t + (int64_t)S * gridDim.x < ntiles)
+                issue_tile(P, it + S, di_issue, smem_base, SB, S, full_bar(s, k + 1));
+        }
     }
 }
 
