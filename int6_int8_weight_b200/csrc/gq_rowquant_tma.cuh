@@ -123,16 +123,21 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
         : "memory");
 }
 
-// Four consecutive elements (quad j) of a row held in shared memory.
+// Four consecutive elements (quad j) of a row held in shared memory.  The
+// shared-memory loads of the row kernels are plain (not volatile) asm, free
+// for the compiler to schedule: every address they take derives from the
+// stage address that the consumer loop launders through a volatile asm after
+// the stage's barrier wait, so none can move above the wait or merge with a
+// load of an earlier fill of the stage.
 template <int DT>
 __device__ __forceinline__ void lds_quad(uint32_t row, int j, float v[4]) {
     if constexpr (DT == kF32) {
-        asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+        asm("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
                      : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3])
                      : "r"(row + 16u * (uint32_t)j));
     } else {
         uint32_t a, b;
-        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(a), "=r"(b) : "r"(row + 8u * (uint32_t)j));
+        asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(a), "=r"(b) : "r"(row + 8u * (uint32_t)j));
         v[0] = __uint_as_float(a << 16);
         v[1] = __uint_as_float(a & 0xFFFF0000u);
         v[2] = __uint_as_float(b << 16);
@@ -339,14 +344,14 @@ __device__ __forceinline__ void topm_scan(uint32_t row, int nq, int tl, int lpr,
         H.init();
         for (; i + 2 <= nfull; i += 2, sa += 2 * step) {
             uint32_t a0, a1, b0, b1;
-            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(a0), "=r"(a1) : "r"(sa));
-            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(b0), "=r"(b1) : "r"(sa + step));
+            asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(a0), "=r"(a1) : "r"(sa));
+            asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(b0), "=r"(b1) : "r"(sa + step));
             H.insert2(as_bf162(a0 & 0x7FFF7FFFu), as_bf162(a1 & 0x7FFF7FFFu));
             H.insert2(as_bf162(b0 & 0x7FFF7FFFu), as_bf162(b1 & 0x7FFF7FFFu));
         }
         for (int j = tl + lpr * i; j < nq; j += lpr, sa += step) {
             uint32_t a0, a1;
-            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(a0), "=r"(a1) : "r"(sa));
+            asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(a0), "=r"(a1) : "r"(sa));
             H.insert2(as_bf162(a0 & 0x7FFF7FFFu), as_bf162(a1 & 0x7FFF7FFFu));
         }
         H.to_f32(L);
@@ -1020,7 +1025,8 @@ rowquant_tma_kernel(const __grid_constant__ TmaParams P) {
         const int64_t r0 = (t - P.start[di]) * D.tile_rows;
         const int nr = (int)min((int64_t)D.tile_rows, D.rows - r0);
         const uint32_t row_bytes = (uint32_t)(D.cols * (D.dtype == kF32 ? 4 : 2));
-        const uint32_t stage = smem_base + (uint32_t)s * SB;
+        uint32_t stage;   // opaque to the compiler, ordered after the wait (see lds_quad)
+        asm volatile("mov.b32 %0, %1;" : "=r"(stage) : "r"(smem_base + (uint32_t)s * SB) : "memory");
         Slot T;
         T.init(lpr, warp, lane);
         const int slots = team_threads >> T.lg;          // slots of this tile-team
