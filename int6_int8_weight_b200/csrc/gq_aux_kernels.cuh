@@ -34,6 +34,7 @@ struct SelParams {
 };
 
 constexpr int kSelBins = 2048;
+constexpr int kSelUnroll = 8;
 
 // PASS 0: digit = key bits 30..20; PASS 1: bits 19..9 among keys whose bits
 // 30..20 equal the chosen prefix; PASS 2: bits 8..0 among keys whose bits
@@ -69,20 +70,42 @@ ptsel_kernel(const __grid_constant__ SelParams P) {
             if ((key >> 9) == prefix) atomicAdd(&h[key & 0x1FFu], 1u);
         }
     };
+    // Contiguous rows with a 16-byte aligned start: 16-byte loads, kSelUnroll
+    // of them in flight per thread before any is counted (the histogram
+    // atomics would otherwise serialize the loads).
     const bool flat = D.ld == D.cols;
-    const bool vec = flat && D.dtype == kF32 && (reinterpret_cast<uintptr_t>(D.w) & 15u) == 0 &&
-                     ((r0 * D.cols) & 3) == 0;
+    const int epv = D.dtype == kF32 ? 4 : 8;                    // elements per 16 bytes
+    const bool vec = flat && (reinterpret_cast<uintptr_t>(D.w) & 15u) == 0 && ((r0 * D.cols) % epv) == 0;
     if (vec) {
-        // contiguous fp32 rows, 16-byte aligned: four elements per thread and step
         const int64_t e0 = r0 * D.cols, e1 = r1 * D.cols;
-        const int64_t n4 = (e1 - e0) >> 2;
-        const float4* src = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(D.w) + e0);
-        for (int64_t i = tid; i < n4; i += kBlockThreads) {
-            const float4 v = src[i];
-            count(v.x); count(v.y); count(v.z); count(v.w);
+        const int64_t nv = (e1 - e0) / epv;
+        const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(D.w) + e0 * esz);
+        auto count16 = [&](const uint4& v) {
+            if (D.dtype == kF32) {
+                count(__uint_as_float(v.x)); count(__uint_as_float(v.y));
+                count(__uint_as_float(v.z)); count(__uint_as_float(v.w));
+            } else {
+                const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    count(__uint_as_float(u[k] << 16));
+                    count(__uint_as_float(u[k] & 0xFFFF0000u));
+                }
+            }
+        };
+        int64_t i = tid;
+        for (; i + (int64_t)(kSelUnroll - 1) * kBlockThreads < nv; i += (int64_t)kSelUnroll * kBlockThreads) {
+            uint4 v[kSelUnroll];
+#pragma unroll
+            for (int u = 0; u < kSelUnroll; ++u) v[u] = src[i + (int64_t)u * kBlockThreads];
+#pragma unroll
+            for (int u = 0; u < kSelUnroll; ++u) count16(v[u]);
         }
-        for (int64_t e = e0 + 4 * n4 + tid; e < e1; e += kBlockThreads)
-            count(reinterpret_cast<const float*>(D.w)[e]);
+        for (; i < nv; i += kBlockThreads) count16(src[i]);
+        const char* wb = reinterpret_cast<const char*>(D.w);
+        for (int64_t e = e0 + nv * epv + tid; e < e1; e += kBlockThreads)
+            count(D.dtype == kF32 ? reinterpret_cast<const float*>(wb)[e]
+                                  : bf16_bits_to_float(reinterpret_cast<const uint16_t*>(wb)[e]));
     } else {
         for (int64_t r = r0; r < r1; ++r) {
             const char* rowp = reinterpret_cast<const char*>(D.w) + r * D.ld * esz;

@@ -233,6 +233,60 @@ def test_ragged_shapes_all_paths(gq, rows, cols, dtype):
     run_train_and_check(gq, w, 8, 0.5, per_tensor=True, what=f"{rows}x{cols} per-tensor train")
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("rows,cols", [(1536, 512), (333, 1000), (700, 97)])
+def test_per_tensor_large_flat(gq, dtype, rows, cols):
+    """Per-tensor groups spanning many select items: the vector loads of the
+    histogram passes (several unrolled trips per thread, then the remainder
+    and a scalar tail) must count every element once."""
+    rng = np.random.default_rng(rows + cols)
+    w = synth.random_matrix(rng, rows, cols, "t3")
+    if dtype == "bf16":
+        w = synth.to_bf16_bits(w).reshape(rows, cols)
+    for p in (0.999, 0.9, 0.5):
+        run_export_and_check(gq, w, 6, p, per_tensor=True, what=f"{rows}x{cols} {dtype} per-tensor p{p}")
+
+
+def _p_for_rank(n, m):
+    """A p whose clip is the m-th largest of n keys, checked with the oracle's rule."""
+    p = (n - m + 1) / n
+    assert oracle.k_from_p(n, p) == n - m + 1
+    return p
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("case", ["zeros", "constant", "three_values", "ties_at_rank", "t3"])
+def test_per_tensor_select_ties_and_tails(gq, dtype, case):
+    """Per-tensor groups with heavy ties (all-zero, all-equal, three values,
+    ties at the selected rank) and sizes that end inside a 16-byte vector,
+    at ranks from 1 to a few thousand: every select pass must count each
+    element once and the tie-breaking must not matter."""
+    rng = np.random.default_rng(len(case) * 17 + (dtype == "bf16"))
+    chunk = 16384 if dtype == "f32" else 32768
+    shapes = [(3, chunk // 3 + 33),            # just over 16 / 32 K elements, odd tail
+              (chunk // 64 + 1, 64 + 3),       # ragged row length
+              (5 * chunk // 512 + 1, 512)]     # several select blocks
+    for rows, cols in shapes:
+        n = rows * cols
+        if case == "zeros":
+            w = np.zeros((rows, cols), np.float32)
+        elif case == "constant":
+            w = np.full((rows, cols), -0.0125, np.float32)
+        elif case == "three_values":
+            w = rng.choice(np.array([0.0, 0.25, -0.5], np.float32), size=(rows, cols))
+        elif case == "ties_at_rank":
+            w = (rng.integers(-3, 4, size=(rows, cols)) * 0.125).astype(np.float32)
+        else:
+            w = synth.random_matrix(rng, rows, cols, "t3")
+        if dtype == "bf16":
+            w = synth.to_bf16_bits(w).reshape(rows, cols)
+        limit = chunk // 4 + 1
+        ranks = sorted({1, 2, min(n, 200), min(n, limit), min(n, limit + 1)})
+        for m in ranks:
+            run_export_and_check(gq, w, 6, _p_for_rank(n, m), per_tensor=True,
+                                 what=f"{case} {dtype} {rows}x{cols} m={m}")
+
+
 @pytest.mark.parametrize("m", [1, 2, 3, 4, 5, 8, 9, 64, 1000])
 @pytest.mark.parametrize("cols", [1536, 4096])
 def test_every_selection_rank(gq, m, cols):
