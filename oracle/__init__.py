@@ -28,6 +28,7 @@ from . import build as _build
 
 OR_OK, OR_ERR_ARG, OR_ERR_RANGE, OR_ERR_NONFINITE, OR_ERR_NOMEM = 0, 1, 2, 3, 4
 F32, BF16 = 0, 1
+AVG_MEAN, AVG_EMA = 0, 1
 
 
 def _ptr(a):
@@ -69,6 +70,8 @@ class Oracle:
         L.or_ste_bwd.restype = i32
         L.or_passthrough_f16.argtypes = [vp, i32, i64, vp]
         L.or_passthrough_f16.restype = i32
+        L.or_average_update.argtypes = [vp, vp, i32, i64, i32, i64, f32]
+        L.or_average_update.restype = i32
         L.or_k_from_p.argtypes = [i64, f64]
         L.or_k_from_p.restype = i64
         L.or_packed_row_bytes.argtypes = [i64, i32]
@@ -137,6 +140,28 @@ class Oracle:
         if st != OR_OK:
             raise ValueError(f"oracle ste status {st}")
         return res
+
+    def average_update(self, avg: np.ndarray, x: np.ndarray, kind: int, count: int = 0,
+                       decay: float = 0.997) -> np.ndarray:
+        """Snapshot averaging (readings R10 / R11 in gq_oracle.c): the new
+        binary32 average after snapshot ``x`` (float32, or bf16 bits as
+        uint16); ``kind`` AVG_MEAN with ``count`` snapshots already in
+        ``avg``, or AVG_EMA with ``decay``."""
+        x = np.ascontiguousarray(x)
+        res = np.array(avg, dtype=np.float32, copy=True).reshape(x.shape)
+        st = self.L.or_average_update(_ptr(res), _ptr(x), _dtype_code(x), x.size, int(kind),
+                                      int(count), float(decay))
+        if st != OR_OK:
+            raise ValueError(f"oracle average status {st}")
+        return res
+
+    def fakequant_average(self, w: np.ndarray, avg: np.ndarray, qbits: int, p: float, kind: int,
+                          count: int = 0, decay: float = 0.997, per_tensor: bool = False,
+                          export: bool = False):
+        """Fake-quant of ``w`` followed by the average update with its output
+        as the snapshot; returns (QuantResult, new average)."""
+        ref = self.quantize(w, qbits, p, per_tensor=per_tensor, export=export)
+        return ref, self.average_update(avg, ref.dq, kind, count, decay)
 
     def passthrough_f16(self, x: np.ndarray) -> np.ndarray:
         """Small-tensor passthrough: binary16 bit patterns (uint16) of ``x``."""

@@ -54,6 +54,15 @@
  *      one binary32 add (bf16: rounded back to nearest even).
  *   R8 bf16 input is widened exactly to binary32 and computed in binary32.
  *   R9 a group holding NaN or +-inf is outside the method; it is reported.
+ *   R10 averaging of quantize-dequantize snapshots ("stochastic quantized
+ *      weight averaging"): a binary32 running average a of snapshots x, the
+ *      fake-quant outputs as the model holds them (bf16 widened exactly).
+ *      Mean (the SWA form): with n snapshots already in a, the next one gives
+ *      a' = a + (x - a) * t, t = 1 / (n + 1), each step one binary32
+ *      operation; n = 0 sets a' = x.
+ *   R11 exponential moving average of the snapshots: a' = d*a + c*x with
+ *      c = 1 - d, each product, the difference and the sum one binary32
+ *      operation (the pages give d = 0.997).
  *
  * Build: plain C11, gcc -O2 -ffp-contract=off, no fast-math, SSE (never x87)
  * binary32 arithmetic, default rounding mode (round to nearest even).
@@ -66,6 +75,7 @@
 enum { OR_OK = 0, OR_ERR_ARG = 1, OR_ERR_RANGE = 2, OR_ERR_NONFINITE = 3,
        OR_ERR_NOMEM = 4 };
 enum { OR_F32 = 0, OR_BF16 = 1 };
+enum { OR_AVG_MEAN = 0, OR_AVG_EMA = 1 };
 
 /* ---------------------------------------------------------------- bits --- */
 
@@ -430,6 +440,54 @@ int or_ste_bwd(const void* g_out, void* g_w, int dtype, int64_t numel,
         }
     }
     return OR_OK;
+}
+
+/* ------------------------------------------------- snapshot averaging --- */
+
+/*
+ * Running average of quantize-dequantize snapshots, in place (R10, R11).
+ * Sources: "Record: Unified Attention + FA3 + Legal TTT" (PR #1202), Novel
+ * Contributions (stochastic quantized weight averaging of
+ * quantize-dequantize snapshots); "SubSixteen v2: Int6 QAT + MLP 3x + SWA +
+ * Sliding Window" (PR #69), Weight Averaging (EMA decay 0.997; SWA every 50
+ * steps after 20 % of training).
+ */
+int or_average_update(float* a, const void* x, int dtype, int64_t numel, int kind,
+                      int64_t count, float decay)
+{
+    if (!a || !x || numel < 0)
+        return OR_ERR_ARG;
+    if (dtype != OR_F32 && dtype != OR_BF16)
+        return OR_ERR_ARG;
+    if (kind == OR_AVG_MEAN) {
+        if (count < 0 || count >= (1 << 24))       /* n + 1 exact in binary32 */
+            return OR_ERR_ARG;
+        float t = 1.0f / (float)(count + 1);
+        for (int64_t i = 0; i < numel; ++i) {
+            float xi = load_elem(x, dtype, i);
+            if (count == 0) {
+                a[i] = xi;
+            } else {
+                float e = xi - a[i];
+                float u = e * t;
+                a[i] = a[i] + u;
+            }
+        }
+        return OR_OK;
+    }
+    if (kind == OR_AVG_EMA) {
+        if (!(decay >= 0.0f && decay <= 1.0f))
+            return OR_ERR_ARG;
+        float c = 1.0f - decay;
+        for (int64_t i = 0; i < numel; ++i) {
+            float xi = load_elem(x, dtype, i);
+            float kept = decay * a[i];
+            float added = c * xi;
+            a[i] = kept + added;
+        }
+        return OR_OK;
+    }
+    return OR_ERR_ARG;
 }
 
 /* Small-tensor passthrough: binary16 round-to-nearest-even of each value. */

@@ -39,6 +39,12 @@ MUTANTS = {
                              "if (r < (float)(-qmax - 1)) r = (float)(-qmax - 1);"),
     "ste_accumulate_drops_term": ("store_elem(g_w, dtype, i, a + b);",
                                   "store_elem(g_w, dtype, i, b);"),
+    "mean_weight_off_by_one": ("float t = 1.0f / (float)(count + 1);",
+                               "float t = 1.0f / (float)(count + 2);"),
+    "mean_first_blended": ("if (count == 0) {", "if (count < 0) {"),
+    "mean_drops_average": ("a[i] = a[i] + u;", "a[i] = u;"),
+    "ema_wrong_factor": ("float added = c * xi;", "float added = decay * xi;"),
+    "ema_sign": ("float c = 1.0f - decay;", "float c = decay - 1.0f;"),
 }
 
 CHECKS = [   # cheapest first: a mutant stops at the first pin that rejects it
@@ -53,6 +59,7 @@ CHECKS = [   # cheapest first: a mutant stops at the first pin that rejects it
     pins.check_torch_round,
     pins.check_invariants,
     pins.check_pack_roundtrip_exhaustive,
+    pins.check_average,
 ]
 
 

@@ -6,7 +6,11 @@
   (torch.kthvalue, torch CPU division + round-half-even, numpy float16,
   torch bfloat16),
 * invariants (|q| <= qmax, clip maps to +-qmax, error bound, pack round trip
-  over every code quadruple, STE identity, dequant == export w_hat).
+  over every code quadruple, STE identity, dequant == export w_hat),
+* snapshot averaging: the first snapshot is copied, and the mean of two
+  snapshots, a mean step with weight 1/4 and an EMA step with decay 1/2
+  equal the exact rational results on dyadic inputs; decay 0 / 1 keep the
+  snapshot / the average; a long EMA of a constant follows 1 - d^k.
 
 The ``orc`` fixture is parametrised so that ``test_oracle_mutants.py`` can run
 the same checks against oracle copies with a planted mistake.
@@ -485,3 +489,70 @@ def test_export_plan_rules():
     assert plan.classify("conv", (64, 32, 3, 3), True, P) == ("fp16", None)
     assert plan.patterns_from_env("a.weight, b ,") == ("a.weight", "b")
     assert plan.patterns_from_env(None) == P
+
+
+# ------------------------------------------------------ snapshot averaging --
+
+def _dyadic(rng, n, lo=-2 ** 10, hi=2 ** 10, shift=8):
+    """Values k / 2^shift with small integers k: sums, halves and quarters of
+    them are exact in binary32."""
+    return (rng.integers(lo, hi, size=n).astype(np.float64) / 2 ** shift).astype(np.float32)
+
+
+def check_average(orc, seed=31):
+    rng = np.random.default_rng(seed)
+    M, E = oracle.AVG_MEAN, oracle.AVG_EMA
+    # the first snapshot replaces whatever the average held (a stale average
+    # of a far larger magnitude would leave a trace if it were blended in)
+    x = rng.standard_normal(257).astype(np.float32)
+    stale = (rng.standard_normal(257) * 1e30).astype(np.float32)
+    a = orc.average_update(stale, x, M, count=0)
+    assert np.array_equal(a.view(np.uint32), x.view(np.uint32))
+    xb = synth.to_bf16_bits(x)
+    a = orc.average_update(stale, xb, M, count=0)
+    assert np.array_equal(a.view(np.uint32), (xb.astype(np.uint32) << 16))
+    # mean of two snapshots, and a mean step with t = 1/4, are exact here
+    x0, x1 = _dyadic(rng, 500), _dyadic(rng, 500)
+    a = orc.average_update(np.zeros(500, np.float32), x0, M, count=0)
+    a = orc.average_update(a, x1, M, count=1)
+    want = [float((Fraction(float(u)) + Fraction(float(v))) / 2) for u, v in zip(x0, x1)]
+    assert np.array_equal(a, np.array(want, np.float32))
+    a3 = _dyadic(rng, 500)
+    a = orc.average_update(a3, x1, M, count=3)
+    want = [float(Fraction(float(u)) + (Fraction(float(v)) - Fraction(float(u))) / 4)
+            for u, v in zip(a3, x1)]
+    assert np.array_equal(a, np.array(want, np.float32))
+    # EMA with decay 1/2 is the exact midpoint; decay 0 keeps the snapshot,
+    # decay 1 the average (non-zero values: the +-0 sums are not at issue)
+    a = orc.average_update(x0, x1, E, decay=0.5)
+    want = [float((Fraction(float(u)) + Fraction(float(v))) / 2) for u, v in zip(x0, x1)]
+    assert np.array_equal(a, np.array(want, np.float32))
+    nz0 = np.where(x0 == 0, np.float32(0.5), x0)
+    nz1 = np.where(x1 == 0, np.float32(0.25), x1)
+    assert np.array_equal(orc.average_update(nz0, nz1, E, decay=0.0), nz1)
+    assert np.array_equal(orc.average_update(nz0, nz1, E, decay=1.0), nz0)
+    # the pages' decay over 300 steps of a constant snapshot: 1 - 0.997^k
+    # (float32 rounding over 300 steps stays far inside 1e-4)
+    a = np.zeros(4, np.float32)
+    one = np.ones(4, np.float32)
+    for _ in range(300):
+        a = orc.average_update(a, one, E, decay=0.997)
+    assert np.all(np.abs(a - (1.0 - 0.997 ** 300)) < 1e-4)
+    # arguments outside the definition are refused
+    for bad in (dict(kind=2), dict(kind=E, decay=1.5), dict(kind=M, count=-1)):
+        with pytest.raises(ValueError):
+            orc.average_update(x0, x1, bad.pop("kind"), **bad)
+
+
+def test_average_pins(orc):
+    check_average(orc)
+
+
+def test_fakequant_average_composes(orc):
+    """The fused reference is the fake-quant output fed to the average."""
+    rng = np.random.default_rng(3)
+    w = synth.random_matrix(rng, 7, 40, "t3")
+    avg = rng.standard_normal((7, 40)).astype(np.float32)
+    ref, a = orc.fakequant_average(w, avg, 6, 0.99, oracle.AVG_MEAN, count=2)
+    assert np.array_equal(a, orc.average_update(avg, ref.dq, oracle.AVG_MEAN, count=2))
+    assert np.array_equal(ref.dq, orc.quantize(w, 6, 0.99, export=False).dq)
