@@ -341,7 +341,18 @@ def measure_rows(gq, device, peak):
     arr = gq._arr([d])
     record("fakequant train bf16 16384^2 int6 absmax",
            timed(lambda: gq.LIB.gq_fakequant_fwd(arr, 1, 0, None, 0, None, None)), 4 * n, 2 * n, 1)
-    del W, o, outd, Wb, dqb
+    # snapshot averaging fused with the training fake-quant (bf16 weights,
+    # binary32 running mean and EMA updated in place; no w_hat written)
+    avg = torch.zeros(16384, 16384, device=device)
+    d0 = gq.GQTensor(w=Wb.data_ptr(), dtype=1, qbits=6, gran=0, reserved=0, rows=16384, cols=16384,
+                     ld=16384, p=1.0, dq=0, codes=0, packed=0, scale_f16=0, scale_f32=0, clip=0)
+    arr0 = gq._arr([d0])
+    for kind, name, count in ((gq.GQ_AVG_MEAN, "mean", 5), (gq.GQ_AVG_EMA, "EMA 0.997", 0)):
+        aa = gq._avg_arr([gq.GQAvg(avg=avg.data_ptr(), kind=kind, decay=0.997, count=count)])
+        record(f"fakequant + snapshot {name} bf16 16384^2 int6 (average only)",
+               timed(lambda: gq.LIB.gq_fakequant_average(arr0, aa, 1, 0, None, 0, None, None)),
+               10 * n, 2 * n, 1, note="reads w (2 B) and the binary32 average (4 B), writes the average (4 B)")
+    del W, o, outd, Wb, dqb, avg
 
     # model-shaped batched workloads (L2-resident: flushed between reps)
     def batch(specs_arrays, export=True, per_tensor_override=None, name="", note=""):

@@ -173,6 +173,46 @@ GQ_API gq_status gq_fakequant_fwd(const gq_tensor* t, int n, gq_scale_mode mode,
                            cudaStream_t stream);
 
 /*
+ * Averaging of quantize-dequantize snapshots (weight averaging of the
+ * fake-quant weights): one binary32 running average per tensor, updated in
+ * the same pass that fake-quantizes the tensor.  The snapshot x is the
+ * fake-quant output w_hat as the model holds it (bf16 w_hat widened
+ * exactly), as gq_fakequant_fwd would write it in the same mode.
+ *   avg    device binary32 [rows, cols], dense, at least 4-byte aligned
+ *          (16-byte aligned rows take the vector path); read and written
+ *   kind   GQ_AVG_MEAN: a' = RN(a + RN(RN(x - a) * t)), t = RN(1 / (count + 1)),
+ *          and count == 0 sets a' = x (the first snapshot);
+ *          GQ_AVG_EMA:  a' = RN(RN(decay * a) + RN(c * x)), c = RN(1 - decay)
+ *   decay  EMA factor in [0, 1]
+ *   count  GQ_AVG_MEAN: snapshots already in avg, 0 <= count < 2^24
+ * Sources: stochastic quantized weight averaging of quantize-dequantize
+ * snapshots ("Record: Unified Attention + FA3 + Legal TTT" page, Novel
+ * Contributions); EMA decay 0.997 and SWA every 50 steps ("SubSixteen v2"
+ * page, Weight Averaging).
+ */
+typedef enum gq_avg_kind { GQ_AVG_MEAN = 0, GQ_AVG_EMA = 1 } gq_avg_kind;
+
+typedef struct gq_avg {
+    float* avg;
+    int32_t kind;
+    float decay;
+    int64_t count;
+} gq_avg;
+
+/*
+ * Fake-quant forward fused with the snapshot average a[i] of t[i]: t[i].dq
+ * is optional (w_hat is written when given); clip, scale_f32 (and scale_f16
+ * in GQ_SCALE_F16 mode) are optional; codes and packed must be NULL.
+ * Argument errors as gq_fakequant_fwd, plus GQ_ERR_INVALID_ARG for a NULL
+ * average of a non-empty tensor, an unknown kind, decay outside [0, 1] or
+ * count outside [0, 2^24), and GQ_ERR_MISALIGNED for an average that is
+ * not 4-byte aligned.
+ */
+GQ_API gq_status gq_fakequant_average(const gq_tensor* t, const gq_avg* a, int n,
+                                      gq_scale_mode mode, void* d_ws, size_t ws_bytes,
+                                      int32_t* d_status, cudaStream_t stream);
+
+/*
  * Straight-through backward: g_w = g_out (accumulate = 0, bitwise copy) or
  * g_w = g_w + g_out (accumulate = 1, one binary32 add, rounded back to bf16
  * for GQ_BF16).  numel elements, dense.  Source: the straight-through

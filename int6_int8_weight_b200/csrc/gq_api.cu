@@ -54,9 +54,20 @@ int64_t packed_row_bytes(int64_t cols, int qbits) {
     return -1;
 }
 
-enum class Op { Select, FakeQuant, Export };
+enum class Op { Select, FakeQuant, Export, Average };
 
 // Validate one descriptor for an operation.  Returns GQ_OK or an error.
+// The running average that goes with a tensor of gq_fakequant_average.
+gq_status check_avg(const gq_tensor& t, const gq_avg& a) {
+    if (a.kind != GQ_AVG_MEAN && a.kind != GQ_AVG_EMA) return GQ_ERR_INVALID_ARG;
+    if (a.kind == GQ_AVG_MEAN && (a.count < 0 || a.count >= (int64_t)1 << 24)) return GQ_ERR_INVALID_ARG;
+    if (a.kind == GQ_AVG_EMA && !(a.decay >= 0.0f && a.decay <= 1.0f)) return GQ_ERR_INVALID_ARG;
+    if (t.rows == 0 || t.cols == 0) return GQ_OK;
+    if (!a.avg) return GQ_ERR_INVALID_ARG;
+    if (!aligned(a.avg, 4)) return GQ_ERR_MISALIGNED;
+    return GQ_OK;
+}
+
 gq_status check_tensor(const gq_tensor& t, Op op, bool f16_mode) {
     if (t.reserved != 0) return GQ_ERR_INVALID_ARG;
     if (t.dtype != GQ_F32 && t.dtype != GQ_BF16) return GQ_ERR_INVALID_ARG;
@@ -83,6 +94,10 @@ gq_status check_tensor(const gq_tensor& t, Op op, bool f16_mode) {
             break;
         case Op::FakeQuant:
             if (!t.dq || t.packed) return GQ_ERR_INVALID_ARG;
+            if (t.scale_f16 && !f16_mode) return GQ_ERR_INVALID_ARG;
+            break;
+        case Op::Average:
+            if (t.codes || t.packed) return GQ_ERR_INVALID_ARG;
             if (t.scale_f16 && !f16_mode) return GQ_ERR_INVALID_ARG;
             break;
         case Op::Export:
@@ -183,6 +198,10 @@ bool tma_eligible(const gq_tensor& T, int32_t flags) {
 // Output configuration of the branch-free loops, or kOutGeneric.
 int32_t tma_out_mode(const RowDesc& D) {
     int32_t mode = 0;
+    if (D.avg) {
+        if (!(D.flags & kVecAvg)) return kOutGeneric;
+        mode |= kOutAvg;
+    }
     if (D.dq) {
         if (!(D.flags & kVecDq)) return kOutGeneric;
         mode |= kOutDq;
@@ -207,6 +226,8 @@ int32_t tma_out_mode(const RowDesc& D) {
         case kOutPacked:
         case kOutDq | kOutCodes | kOutPacked | kOutSix:
         case kOutDq | kOutCodes:
+        case kOutAvg:
+        case kOutDq | kOutAvg:
             return mode;
         default:
             return kOutGeneric;
@@ -291,11 +312,14 @@ gq_status run_passthrough(const std::vector<PassDesc>& pd, cudaStream_t stream) 
 
 // The shared driver of gq_row_clip_select, gq_fakequant_fwd and gq_export_pack.
 gq_status quantize_batch(const gq_tensor* t, int n, Op op, bool f16_mode, void* ws,
-                         size_t ws_bytes, int32_t* d_status, cudaStream_t stream) {
+                         size_t ws_bytes, int32_t* d_status, cudaStream_t stream,
+                         const gq_avg* avg = nullptr) {
     if (n < 0 || (n > 0 && !t)) return GQ_ERR_INVALID_ARG;
+    if (op == Op::Average && n > 0 && !avg) return GQ_ERR_INVALID_ARG;
     for (int i = 0; i < n; ++i) {
         gq_status st = check_tensor(t[i], op, f16_mode);
         if (st != GQ_OK) return st;
+        if (op == Op::Average && (st = check_avg(t[i], avg[i])) != GQ_OK) return st;
     }
     const size_t need = workspace_size(t, n);
     if (need > 0) {
@@ -335,7 +359,7 @@ gq_status quantize_batch(const gq_tensor* t, int n, Op op, bool f16_mode, void* 
         D.dq = T.dq;
         D.codes = T.codes;
         D.packed = T.packed;
-        D.sf16 = (op == Op::FakeQuant && !f16_mode) ? nullptr : T.scale_f16;
+        D.sf16 = ((op == Op::FakeQuant || op == Op::Average) && !f16_mode) ? nullptr : T.scale_f16;
         D.sf32 = T.scale_f32;
         D.clip_out = T.clip;
         D.status = status;
@@ -347,8 +371,21 @@ gq_status quantize_batch(const gq_tensor* t, int n, Op op, bool f16_mode, void* 
         D.dtype = T.dtype;
         D.qbits = T.qbits;
         D.export_mode = (op == Op::Export || f16_mode) ? 1 : 0;
-        const bool elem = T.dq || T.codes || T.packed;
+        if (op == Op::Average) {
+            const gq_avg& A = avg[i];
+            D.avg = A.avg;
+            if (A.kind == GQ_AVG_MEAN) {
+                D.avg_kind = A.count == 0 ? kAvgCopy : kAvgMean;
+                D.avg_t = 1.0f / (float)(A.count + 1);      // one binary32 division
+            } else {
+                D.avg_kind = kAvgEma;
+                D.avg_t = A.decay;
+                D.avg_c = 1.0f - A.decay;                   // one binary32 subtraction
+            }
+        }
+        const bool elem = T.dq || T.codes || T.packed || D.avg;
         int32_t flags = elem ? kElemOut : 0;
+        if (D.avg && aligned(D.avg, 16) && (T.cols % 4) == 0) flags |= kVecAvg;
         const size_t vin = T.dtype == GQ_F32 ? 16 : 8;
         if (aligned(T.w, vin) && ((T.ld * esz) % (int64_t)vin) == 0) flags |= kVecIn;
         if (T.dq && aligned(T.dq, vin) && ((T.cols * esz) % (int64_t)vin) == 0) flags |= kVecDq;
@@ -436,6 +473,12 @@ gq_status gq_fakequant_fwd(const gq_tensor* t, int n, gq_scale_mode mode, void* 
     if (mode != GQ_SCALE_F32 && mode != GQ_SCALE_F16) return GQ_ERR_INVALID_ARG;
     return quantize_batch(t, n, Op::FakeQuant, mode == GQ_SCALE_F16, d_ws, ws_bytes, d_status,
                           stream);
+}
+
+gq_status gq_fakequant_average(const gq_tensor* t, const gq_avg* avg, int n, gq_scale_mode mode,
+                               void* d_ws, size_t ws_bytes, int32_t* d_status, cudaStream_t stream) {
+    if (mode != GQ_SCALE_F32 && mode != GQ_SCALE_F16) return GQ_ERR_INVALID_ARG;
+    return quantize_batch(t, n, Op::Average, mode == GQ_SCALE_F16, d_ws, ws_bytes, d_status, stream, avg);
 }
 
 gq_status gq_export_pack(const gq_tensor* t, int n, void* d_ws, size_t ws_bytes,

@@ -4,8 +4,10 @@
 // Arithmetic contract (the definitions in include/gq.h): every floating-point
 // step that decides an output bit is one correctly rounded binary32 operation,
 // written with the explicit-rounding intrinsics (__fmul_rn, __fadd_rn,
-// __fdiv_rn, __frcp_rn) or the paired .rn f32x2 instructions (two independent
-// binary32 lanes), so the compiler cannot contract or reassociate it.
+// __fdiv_rn, __frcp_rn), so the compiler cannot contract or reassociate it.
+// The one exception is the reciprocal quotient of the fused row kernel, on
+// paired f32x2 instructions that the code generator may contract: its code
+// is decided by a guard whose margin covers either form (see round8_fast).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -54,6 +56,25 @@ __device__ __forceinline__ uint16_t float_to_bf16_bits(float x) {
 // |x| as an ordered key: non-negative binary32 values order like their bits.
 __device__ __forceinline__ uint32_t abs_key(float x) {
     return __float_as_uint(x) & 0x7FFFFFFFu;
+}
+
+// Running average of quantize-dequantize snapshots (one binary32 array per
+// tensor): kind 0 none, 1 copy (the first snapshot), 2 mean
+// a + (x - a) * t with t = RN(1 / (n + 1)), 3 EMA RN(t * a) + RN(c * x) with
+// t = decay and c = RN(1 - decay).  x is the snapshot as the model holds it.
+constexpr int kAvgNone = 0, kAvgCopy = 1, kAvgMean = 2, kAvgEma = 3;
+
+struct AvgOp {
+    float* a;     // this row's averages (null: no average)
+    float t;
+    float c;
+    int kind;
+};
+
+__device__ __forceinline__ float avg_update(float a, float x, const AvgOp& A) {
+    if (A.kind == kAvgCopy) return x;
+    if (A.kind == kAvgMean) return __fadd_rn(a, __fmul_rn(__fsub_rn(x, a), A.t));
+    return __fadd_rn(__fmul_rn(A.t, a), __fmul_rn(A.c, x));
 }
 
 // Per-group quantization constants.

@@ -41,7 +41,10 @@ struct RowDesc {
     int32_t tile_rows;         // pipelined kernel: rows per shared-memory tile
     int32_t lanes_per_row;     // pipelined kernel: threads per row (8 .. 512)
     int32_t out_mode;          // pipelined kernel: output configuration, -1 generic
-    int32_t pad2;
+    int32_t avg_kind;          // kAvg*: running average of the w_hat snapshots
+    float* avg;                // binary32 [rows, cols] averages (dense), or null
+    float avg_t;               // mean: RN(1 / (n + 1)); EMA: decay
+    float avg_c;               // EMA: RN(1 - decay)
 };
 
 constexpr int32_t kVecIn = 1;       // rows of w are 16-byte (f32) / 8-byte (bf16) aligned
@@ -49,7 +52,8 @@ constexpr int32_t kVecDq = 2;       // rows of dq likewise
 constexpr int32_t kVecCodes = 4;    // rows of codes 4-byte aligned
 constexpr int32_t kVecPacked = 8;   // rows of packed 4-byte aligned
 constexpr int32_t kPerTensor = 16;
-constexpr int32_t kElemOut = 32;    // dq, codes or packed requested
+constexpr int32_t kElemOut = 32;    // dq, codes, packed or an average requested
+constexpr int32_t kVecAvg = 64;     // rows of the average 16-byte aligned
 
 struct RowParams {
     int32_t ndesc;
@@ -235,6 +239,19 @@ __device__ void quantize_row(const RowDesc& D, int64_t r, const Scale& S, int tw
         for (int i = 0; i < 4; ++i) {
             b[i] = quantize_offset(v[i], S);
             q[i] = offset_to_code(b[i]);
+        }
+        if (valid && D.avg) {
+            // the snapshot as the model holds it: bf16 w_hat widened
+            float* arow = D.avg + r * n;
+            const AvgOp A{arow, D.avg_t, D.avg_c, D.avg_kind};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                if (e0 + i < n) {
+                    float x = offset_to_dq(b[i], S);
+                    if (D.dtype != kF32) x = bf16_bits_to_float(float_to_bf16_bits(x));
+                    arow[e0 + i] = avg_update(arow[e0 + i], x, A);
+                }
+            }
         }
         if (valid && dqrow) {
             float d[4];

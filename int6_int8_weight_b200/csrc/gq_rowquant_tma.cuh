@@ -41,7 +41,7 @@ constexpr unsigned long long kWaitLimitNs = 4000000000ull;   // 4 s
 
 // Output configurations with a branch-free inner loop (vector stores
 // guaranteed by the host); anything else takes the generic loop.
-constexpr int kOutDq = 1, kOutCodes = 2, kOutPacked = 4, kOutSix = 8;
+constexpr int kOutDq = 1, kOutCodes = 2, kOutPacked = 4, kOutSix = 8, kOutAvg = 16;
 constexpr int kOutGeneric = -1;
 
 struct TmaParams {
@@ -167,8 +167,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// Two binary32 lanes in one 64-bit register for the paired f32x2 operations
-// (each lane one correctly rounded binary32 operation).
+// Two binary32 lanes in one 64-bit register for the paired f32x2 operations.
+// Each lane is a correctly rounded binary32 operation, but the code generator
+// may contract a paired product with a following paired sum into one fused
+// multiply-add (observed on sm_100a even with contraction disabled), so they
+// serve only where a result does not depend on that (the guarded quotient).
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
     uint64_t r;
     asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
@@ -524,9 +527,13 @@ __device__ __forceinline__ void round8(const float x[8], const Scale& S, float n
 // Rounded quotients of two quads for the branch-free loop: n[k] (integer-
 // valued floats) and b[k] = kMagic + n[k] (the code bits), with one warp
 // vote for both rare events: a quotient within 2^-13 of a half-integer
-// (exact division for that lane) and, with CLAMP, a code beyond qmax.  The
-// products and sums run on element pairs (f32x2), each lane of which is the
-// same correctly rounded binary32 operation as the scalar form.
+// (exact division for that lane) and, with CLAMP, a code beyond qmax.
+// The products and sums run on element pairs (f32x2).  Whether or not the
+// code generator fuses P = x * rcp into the magic sum and into the residual,
+// n is rint(P) or rint(RN(P)) and e is within 2^-24 |P - n| of P - n or of
+// RN(P) - n.  With Q = RN(x / s): |P - Q| < 2^-15 and |RN(P) - P| < 2^-16
+// (|x / s| < 256), so |e| <= 0.5 - 2^-13 gives |Q - n| < 0.5, i.e. n = rint(Q)
+// exactly, and otherwise the lane takes the exact division.
 template <bool CLAMP>
 __device__ __forceinline__ void round8_fast(const float x[8], float rcp, float s, float qmaxf, float n[8],
                                             float b[8]) {
@@ -566,26 +573,51 @@ __device__ __forceinline__ void round8_fast(const float x[8], float rcp, float s
 // turns the sum of four code words b into the biased 24-bit group.
 constexpr uint32_t kSixBias = 0x1ABDF7E0u;
 
+// New averages of a quad.  Scalar explicit-rounding operations: every step
+// must round on its own here (the paired f32x2 forms may be contracted into
+// fused multiply-adds by the code generator).
+__device__ __forceinline__ float4 avg_quad(const float4 a, const float x[4], const AvgOp& A) {
+    return make_float4(avg_update(a.x, x[0], A), avg_update(a.y, x[1], A), avg_update(a.z, x[2], A),
+                       avg_update(a.w, x[3], A));
+}
+
 // Stores of one quad for a compile-time output configuration, at running
 // pointers: pd (w_hat quad), pc (4 code bytes), pp (int8: 4 bytes; int6: this
-// lane's 32-bit word of its 4-lane group, unused by the group's 4th lane).
+// lane's 32-bit word of its 4-lane group, unused by the group's 4th lane), pa
+// (the quad's averages, whose old values a4 the caller loaded early).
 // b[i] = kMagic + q[i]: its low byte is q's two's-complement byte and its low
 // six bits the int6 field.
 template <int DT, int OUT>
-__device__ __forceinline__ void put_quad(char* pd, int8_t* pc, uint8_t* pp, bool valid, int sub,
-                                         const float q[4], const float b[4], float s) {
+__device__ __forceinline__ void put_quad(char* pd, int8_t* pc, uint8_t* pp, float* pa, float4 a4,
+                                         const AvgOp& A, bool valid, int sub, const float q[4],
+                                         const float b[4], float s) {
     const uint32_t b0 = __float_as_uint(b[0]), b1 = __float_as_uint(b[1]);
     const uint32_t b2 = __float_as_uint(b[2]), b3 = __float_as_uint(b[3]);
-    if constexpr ((OUT & kOutDq) != 0) {
+    if constexpr ((OUT & (kOutDq | kOutAvg)) != 0) {
         float w[4];
         const uint64_t S2 = f2_pack(s, s);
         f2_unpack(f2_mul(f2_pack(q[0], q[1]), S2), w[0], w[1]);
         f2_unpack(f2_mul(f2_pack(q[2], q[3]), S2), w[2], w[3]);
-        if constexpr (DT == kF32) {
-            if (valid) *reinterpret_cast<float4*>(pd) = make_float4(w[0], w[1], w[2], w[3]);
-        } else {
-            const uint2 d = make_uint2(pack_bf16x2(w[0], w[1]), pack_bf16x2(w[2], w[3]));
-            if (valid) *reinterpret_cast<uint2*>(pd) = d;
+        uint2 d;
+        if constexpr (DT == kBF16) d = make_uint2(pack_bf16x2(w[0], w[1]), pack_bf16x2(w[2], w[3]));
+        if constexpr ((OUT & kOutDq) != 0) {
+            if constexpr (DT == kF32) {
+                if (valid) *reinterpret_cast<float4*>(pd) = make_float4(w[0], w[1], w[2], w[3]);
+            } else {
+                if (valid) *reinterpret_cast<uint2*>(pd) = d;
+            }
+        }
+        if constexpr ((OUT & kOutAvg) != 0) {
+            // the snapshot as the model holds it: RN(q * s), bf16 w_hat widened
+            float x[4] = {__fmul_rn(q[0], s), __fmul_rn(q[1], s), __fmul_rn(q[2], s), __fmul_rn(q[3], s)};
+            if constexpr (DT == kBF16) {
+                x[0] = __uint_as_float(d.x << 16);
+                x[1] = __uint_as_float(d.x & 0xFFFF0000u);
+                x[2] = __uint_as_float(d.y << 16);
+                x[3] = __uint_as_float(d.y & 0xFFFF0000u);
+            }
+            const float4 r = avg_quad(a4, x, A);
+            if (valid) *reinterpret_cast<float4*>(pa) = r;
         }
     }
     if constexpr ((OUT & kOutCodes) != 0 || ((OUT & kOutPacked) != 0 && (OUT & kOutSix) == 0)) {
@@ -621,18 +653,14 @@ __device__ __forceinline__ void put_quad(char* pd, int8_t* pc, uint8_t* pp, bool
 template <int DT, int OUT, bool CLAMP>
 __device__ __forceinline__ void quantize_row_fast(uint32_t row, int nq, int tl, int lpr, int lg, bool rv,
                                                   float s, float rcp, float qmaxf, char* dq, int8_t* codes,
-                                                  uint8_t* packed) {
+                                                  uint8_t* packed, const AvgOp& A) {
     constexpr uint32_t QB = DT == kF32 ? 16u : 8u;
     constexpr int DQB = DT == kF32 ? 16 : 8;
     constexpr bool SIX = (OUT & kOutSix) != 0;
-    Scale S;
-    S.c = 0.f;
-    S.s = s;
-    S.rcp = rcp;
-    S.qmaxf = qmaxf;
-    S.fast = true;
-    S.zero = false;
+    constexpr bool AVG = (OUT & kOutAvg) != 0;
     const int sub = tl & 3;
+    float* pa = AVG ? A.a + 4 * tl : nullptr;          // averages: 16 bytes per quad
+    const int sa4 = 4 * lpr;
     const uint32_t step = QB * (uint32_t)lpr;
     uint32_t sa = row + QB * (uint32_t)tl;
     char* pd = dq + DQB * tl;
@@ -645,28 +673,37 @@ __device__ __forceinline__ void quantize_row_fast(uint32_t row, int nq, int tl, 
         float x[8];
         lds_quad<DT>(sa, 0, x);
         lds_quad<DT>(sa + step, 0, x + 4);
+        float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+        if (AVG && rv) {                               // issued before the arithmetic
+            a0 = *reinterpret_cast<const float4*>(pa);
+            a1 = *reinterpret_cast<const float4*>(pa + sa4);
+        }
         // only codes of |w| > c can exceed qmax, so the clamp is a rare path
         float q[8], b[8];
         round8_fast<CLAMP>(x, rcp, s, qmaxf, q, b);
-        put_quad<DT, OUT>(pd, pc, pp, rv, sub, q, b, s);
-        put_quad<DT, OUT>(pd + sd, pc + sc, pp + sp, rv, sub, q + 4, b + 4, s);
+        put_quad<DT, OUT>(pd, pc, pp, pa, a0, A, rv, sub, q, b, s);
+        put_quad<DT, OUT>(pd + sd, pc + sc, pp + sp, AVG ? pa + sa4 : nullptr, a1, A, rv, sub, q + 4, b + 4, s);
         sa += 2 * step;
         pd += 2 * sd;
         pc += 2 * sc;
         pp += 2 * sp;
+        if (AVG) pa += 2 * sa4;
     }
     const int niter = (nq + lpr - 1) >> lg;
     for (; i < niter; ++i) {
         const bool valid = rv && (tl + lpr * i < nq);
         float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         if (valid) lds_quad<DT>(sa, 0, x);
+        float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (AVG && valid) a0 = *reinterpret_cast<const float4*>(pa);
         float q[8], b[8];
         round8_fast<CLAMP>(x, rcp, s, qmaxf, q, b);
-        put_quad<DT, OUT>(pd, pc, pp, valid, sub, q, b, s);
+        put_quad<DT, OUT>(pd, pc, pp, pa, a0, A, valid, sub, q, b, s);
         sa += step;
         pd += sd;
         pc += sc;
         pp += sp;
+        if (AVG) pa += sa4;
     }
 }
 
@@ -676,7 +713,8 @@ template <int DT>
 __device__ __forceinline__ void quantize_row_generic(uint32_t row, int nq, int tl, int lpr, bool rv, float c,
                                                   float s, float rcp, float qmaxf, bool fast, bool zero,
                                                   bool clip, bool clamp, char* dq, int8_t* codes,
-                                                  uint8_t* packed, bool vdq, bool vcodes, bool vpk, bool six) {
+                                                  uint8_t* packed, bool vdq, bool vcodes, bool vpk, bool six,
+                                                  const AvgOp& A) {
     Scale S;
     S.c = c;
     S.s = s;
@@ -721,6 +759,15 @@ __device__ __forceinline__ void quantize_row_generic(uint32_t row, int nq, int t
             b[k] = __fadd_rn(q[k], kMagic);
         }
         const int e0 = 4 * j;
+        if (valid && A.a) {
+            // the snapshot as the model holds it (bf16 w_hat widened)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                float x = __fmul_rn(q[k], S.s);
+                if (DT == kBF16) x = bf16_bits_to_float(float_to_bf16_bits(x));
+                A.a[e0 + k] = avg_update(A.a[e0 + k], x, A);
+            }
+        }
         if (valid && dq) {
             float d[4];
 #pragma unroll
@@ -788,10 +835,11 @@ __device__ __forceinline__ void quantize_row_generic(uint32_t row, int nq, int t
 
 template <int DT, int OUT>
 __device__ __forceinline__ void dispatch_fast(bool clamp, uint32_t row, int nq, int tl, int lpr, bool rv,
-                                              const Scale& S, char* dq, int8_t* codes, uint8_t* packed) {
+                                              const Scale& S, char* dq, int8_t* codes, uint8_t* packed,
+                                              const AvgOp& A) {
     const int lg = 31 - __clz(lpr);
-    if (clamp) quantize_row_fast<DT, OUT, true>(row, nq, tl, lpr, lg, rv, S.s, S.rcp, S.qmaxf, dq, codes, packed);
-    else quantize_row_fast<DT, OUT, false>(row, nq, tl, lpr, lg, rv, S.s, S.rcp, S.qmaxf, dq, codes, packed);
+    if (clamp) quantize_row_fast<DT, OUT, true>(row, nq, tl, lpr, lg, rv, S.s, S.rcp, S.qmaxf, dq, codes, packed, A);
+    else quantize_row_fast<DT, OUT, false>(row, nq, tl, lpr, lg, rv, S.s, S.rcp, S.qmaxf, dq, codes, packed, A);
 }
 
 // Quantize + outputs of one row; `rv` false for an idle sub-warp slot (it
@@ -804,6 +852,7 @@ __device__ __forceinline__ void quantize_row(const RowDesc& D, int64_t r, uint32
     char* dq = D.dq ? reinterpret_cast<char*>(D.dq) + r * D.cols * esz : nullptr;
     int8_t* codes = D.codes ? D.codes + r * D.cols : nullptr;
     uint8_t* packed = D.packed ? D.packed + r * D.prb : nullptr;
+    const AvgOp A{D.avg ? D.avg + r * D.cols : nullptr, D.avg_t, D.avg_c, D.avg_kind};
     // a warp takes the branch-free loop only if every row it holds can; the
     // clamp decision must agree too (it is a template parameter there)
     const bool fast_row = out != kOutGeneric && R.S.fast && !R.S.zero && !R.clip;
@@ -812,24 +861,28 @@ __device__ __forceinline__ void quantize_row(const RowDesc& D, int64_t r, uint32
     if (!all_fast) {
         quantize_row_generic<DT>(row, nq, T.tl, T.lpr, rv, R.S.c, R.S.s, R.S.rcp, R.S.qmaxf, R.S.fast, R.S.zero,
                                  R.clip, R.clamp, dq, codes, packed, (D.flags & kVecDq) != 0,
-                                 (D.flags & kVecCodes) != 0, (D.flags & kVecPacked) != 0, D.qbits == 6);
+                                 (D.flags & kVecCodes) != 0, (D.flags & kVecPacked) != 0, D.qbits == 6, A);
         return;
     }
     switch (out) {
         case kOutDq | kOutPacked | kOutSix:
-            dispatch_fast<DT, kOutDq | kOutPacked | kOutSix>(any_clamp, row, nq, T.tl, T.lpr, rv, R.S, dq, codes, packed); break;
+            dispatch_fast<DT, kOutDq | kOutPacked | kOutSix>(any_clamp, row, nq, T.tl, T.lpr, rv, R.S, dq, codes, packed, A); break;
         case kOutDq | kOutPacked:
-            dispatch_fast<DT, kOutDq | kOutPacked>(any_clamp, row, nq, T.tl, T.lpr, rv, R.S, dq, codes, packed); break;
+            dispatch_fast<DT, kOutDq | kOutPacked>(any_clamp, row, nq, T.tl, T.lpr, rv, R.S, dq, codes, packed, A); break;
         case kOutDq:
-            dispatch_fast<DT, kOutDq>(any_clamp, row, nq, T.tl, T.lpr, rv, R.S, dq, codes, packed); break;
+            dispatch_fast<DT, kOutDq>(any_clamp, row, nq, T.tl, T.lpr, rv, R.S, dq, codes, packed, A); break;
         case kOutPacked | kOutSix:
-            dispatch_fast<DT, kOutPacked | kOutSix>(any_clamp, row, nq, T.tl, T.lpr, rv, R.S, dq, codes, packed); break;
+            dispatch_fast<DT, kOutPacked | kOutSix>(any_clamp, row, nq, T.tl, T.lpr, rv, R.S, dq, codes, packed, A); break;
         case kOutPacked:
-            dispatch_fast<DT, kOutPacked>(any_clamp, row, nq, T.tl, T.lpr, rv, R.S, dq, codes, packed); break;
+            dispatch_fast<DT, kOutPacked>(any_clamp, row, nq, T.tl, T.lpr, rv, R.S, dq, codes, packed, A); break;
         case kOutDq | kOutCodes | kOutPacked | kOutSix:
-            dispatch_fast<DT, kOutDq | kOutCodes | kOutPacked | kOutSix>(any_clamp, row, nq, T.tl, T.lpr, rv, R.S, dq, codes, packed); break;
+            dispatch_fast<DT, kOutDq | kOutCodes | kOutPacked | kOutSix>(any_clamp, row, nq, T.tl, T.lpr, rv, R.S, dq, codes, packed, A); break;
+        case kOutAvg:
+            dispatch_fast<DT, kOutAvg>(any_clamp, row, nq, T.tl, T.lpr, rv, R.S, dq, codes, packed, A); break;
+        case kOutDq | kOutAvg:
+            dispatch_fast<DT, kOutDq | kOutAvg>(any_clamp, row, nq, T.tl, T.lpr, rv, R.S, dq, codes, packed, A); break;
         default:
-            dispatch_fast<DT, kOutDq | kOutCodes>(any_clamp, row, nq, T.tl, T.lpr, rv, R.S, dq, codes, packed); break;
+            dispatch_fast<DT, kOutDq | kOutCodes>(any_clamp, row, nq, T.tl, T.lpr, rv, R.S, dq, codes, packed, A); break;
     }
 }
 

@@ -29,7 +29,8 @@ GQ_OK = 0
 GQ_F32, GQ_BF16 = 0, 1
 GQ_PER_ROW, GQ_PER_TENSOR = 0, 1
 GQ_SCALE_F32, GQ_SCALE_F16 = 0, 1
-GQ_STATUS_NONFINITE, GQ_STATUS_RANGE = 1, 2
+GQ_STATUS_NONFINITE, GQ_STATUS_RANGE, GQ_STATUS_TIMEOUT = 1, 2, 4
+GQ_AVG_MEAN, GQ_AVG_EMA = 0, 1
 GQ_KIND_RAW, GQ_KIND_FP16, GQ_KIND_INT8, GQ_KIND_INT6 = 0, 1, 2, 3
 KIND_NAMES = {GQ_KIND_RAW: "raw", GQ_KIND_FP16: "fp16", GQ_KIND_INT8: "int8", GQ_KIND_INT6: "int6"}
 
@@ -37,7 +38,7 @@ STATUS_NAMES = {0: "GQ_OK", 1: "GQ_ERR_INVALID_ARG", 2: "GQ_ERR_UNSUPPORTED",
                 3: "GQ_ERR_MISALIGNED", 4: "GQ_ERR_WORKSPACE", 5: "GQ_ERR_RANGE",
                 6: "GQ_ERR_NONFINITE", 7: "GQ_ERR_CUDA", 8: "GQ_ERR_TIMEOUT"}
 
-EXPORTED = ("gq_row_clip_select", "gq_fakequant_fwd", "gq_ste_bwd", "gq_export_pack",
+EXPORTED = ("gq_row_clip_select", "gq_fakequant_fwd", "gq_fakequant_average", "gq_ste_bwd", "gq_export_pack",
             "gq_export_pack_noalloc", "gq_dequant", "gq_workspace_size", "gq_packed_row_bytes", "gq_k_from_p",
             "gq_plan_kind", "gq_status_string", "gq_last_cuda_error", "gq_last_cuda_error_string")
 
@@ -59,6 +60,10 @@ class GQTensor(C.Structure):
     ]
 
 
+class GQAvg(C.Structure):
+    _fields_ = [("avg", C.c_void_p), ("kind", C.c_int32), ("decay", C.c_float), ("count", C.c_int64)]
+
+
 def _load() -> C.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
@@ -69,11 +74,13 @@ def _load() -> C.CDLL:
     T = C.POINTER(GQTensor)
     L.gq_row_clip_select.argtypes = [T, i32, vp, sz, vp, vp]
     L.gq_fakequant_fwd.argtypes = [T, i32, i32, vp, sz, vp, vp]
+    L.gq_fakequant_average.argtypes = [T, C.POINTER(GQAvg), i32, i32, vp, sz, vp, vp]
     L.gq_export_pack.argtypes = [T, i32, vp, sz, vp, vp]
     L.gq_export_pack_noalloc.argtypes = [T, i32, vp, vp]
     L.gq_ste_bwd.argtypes = [vp, vp, i32, i64, i32, vp]
     L.gq_dequant.argtypes = [vp, vp, i32, i32, i64, i64, vp, i32, vp]
-    for f in ("gq_row_clip_select", "gq_fakequant_fwd", "gq_export_pack", "gq_export_pack_noalloc",
+    for f in ("gq_row_clip_select", "gq_fakequant_fwd", "gq_fakequant_average", "gq_export_pack",
+              "gq_export_pack_noalloc",
               "gq_ste_bwd", "gq_dequant"):
         getattr(L, f).restype = i32
     L.gq_workspace_size.argtypes = [T, i32]
@@ -127,6 +134,18 @@ def gq_row_clip_select(descs, ws=0, ws_bytes=0, d_status=0, stream=None):
 def gq_fakequant_fwd(descs, mode, ws=0, ws_bytes=0, d_status=0, stream=None):
     _check(LIB.gq_fakequant_fwd(_arr(descs), len(descs), mode, ws or None, ws_bytes,
                                 d_status or None, _stream(stream)), "gq_fakequant_fwd")
+
+
+def _avg_arr(avgs):
+    arr = (GQAvg * max(1, len(avgs)))()
+    for i, a in enumerate(avgs):
+        arr[i] = a
+    return arr
+
+
+def gq_fakequant_average(descs, avgs, mode, ws=0, ws_bytes=0, d_status=0, stream=None):
+    _check(LIB.gq_fakequant_average(_arr(descs), _avg_arr(avgs), len(descs), mode, ws or None, ws_bytes,
+                                    d_status or None, _stream(stream)), "gq_fakequant_average")
 
 
 def gq_export_pack(descs, ws=0, ws_bytes=0, d_status=0, stream=None):
@@ -284,7 +303,7 @@ class _Scratch:
 _SCRATCH = _Scratch()
 
 
-def _run(fn_name, reqs, export, mode=None, stream=None, check_status=True):
+def _run(fn_name, reqs, export, mode=None, stream=None, check_status=True, avgs=None):
     if not reqs:
         return []
     descs, outs = _prepare(reqs, export)
@@ -296,6 +315,8 @@ def _run(fn_name, reqs, export, mode=None, stream=None, check_status=True):
                 stream=stream)
     if fn_name == "fakequant":
         gq_fakequant_fwd(descs, mode, **args)
+    elif fn_name == "average":
+        gq_fakequant_average(descs, avgs, mode, **args)
     elif fn_name == "export":
         gq_export_pack(descs, **args)
     else:
@@ -310,6 +331,21 @@ def _run(fn_name, reqs, export, mode=None, stream=None, check_status=True):
 def fakequant(reqs, mode=GQ_SCALE_F32, stream=None, check_status=True):
     """Batched STE fake-quant forward (one launch for the batch)."""
     return _run("fakequant", reqs, False, mode, stream, check_status)
+
+
+def fakequant_average(reqs, averages, kind=GQ_AVG_MEAN, count=0, decay=0.997, mode=GQ_SCALE_F32,
+                      stream=None, check_status=True):
+    """Fake-quant of each request fused with the update of its running
+    average of quantize-dequantize snapshots (``averages``: float32 tensors
+    of the weights' shape, updated in place).  ``kind`` GQ_AVG_MEAN with
+    ``count`` snapshots already averaged, or GQ_AVG_EMA with ``decay``.
+    w_hat is returned only for requests with ``want_dq``."""
+    avgs = []
+    for r, a in zip(reqs, averages, strict=True):
+        if a.dtype != torch.float32 or not a.is_contiguous() or a.shape != r.w.shape:
+            raise ValueError("averages are contiguous float32 tensors of the weight's shape")
+        avgs.append(GQAvg(avg=a.data_ptr(), kind=kind, decay=float(decay), count=int(count)))
+    return _run("average", reqs, False, mode, stream, check_status, avgs)
 
 
 def export_pack(reqs, stream=None, check_status=True):
