@@ -275,6 +275,29 @@ GQ_API gq_status gq_dequant(const uint8_t* d_packed, const uint16_t* d_scale_f16
                      int qbits, gq_gran gran, int64_t rows, int64_t cols,
                      void* d_out, gq_dtype out_dtype, cudaStream_t stream);
 
+/*
+ * The consuming GEMM with the dequant in its weight load:
+ *   Y[m, n] = sum_k X[m, k] * W_hat[n, k],  W_hat[n, k] = bf16(RN(q[n, k] * s[n]))
+ * with q the int6 / int8 codes of row n in d_packed (rows of
+ * gq_packed_row_bytes(K, qbits) bytes, as gq_export_pack writes them for a
+ * weight [N, K] exported per row) and s[n] = (float)scale_f16[n].  W_hat is
+ * the bf16 fake-quant weight the forward pass would multiply by; it is
+ * rebuilt tile by tile in shared memory and never written to memory.
+ *   d_x      bf16 [M, ldx] activations, row-major, 16-byte aligned, ldx % 8 == 0
+ *   d_y      fp32 [M, ldy] output, overwritten; 16-byte aligned, ldy % 4 == 0
+ *   d_status nullable: GQ_STATUS_TIMEOUT if a bounded wait on the device gave up
+ * Products are exact (bf16 x bf16) and accumulate in binary32 in the tensor
+ * cores' order, so Y is not bitwise reproducible against a sequential sum:
+ * |Y - exact| <= (K/8 + 4) * 2^-24 * sum_k |X[m, k] * W_hat[n, k]|.
+ * K must be a multiple of 64 (GQ_ERR_UNSUPPORTED otherwise).  Source: STE
+ * fake quantization in the forward pass whose weights feed the layer's
+ * matmuls ("SubSixteen v2" page, Other; PR #1202, Quantization), with the
+ * int6 / int8 storage of the export (PR #1495, Mixed-bit quantization).
+ */
+GQ_API gq_status gq_gemm_dequant(const void* d_x, int64_t M, int64_t K, int64_t ldx, const uint8_t* d_packed,
+                                 const uint16_t* d_scale_f16, int qbits, int64_t N, float* d_y, int64_t ldy,
+                                 int32_t* d_status, cudaStream_t stream);
+
 /* Device workspace bytes a batch needs (0 when it has no per-tensor group). */
 GQ_API size_t gq_workspace_size(const gq_tensor* t, int n);
 

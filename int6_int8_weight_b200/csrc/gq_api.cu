@@ -11,7 +11,10 @@
 #include <vector>
 
 #include "gq.h"
+#include <cudaTypedefs.h>
+
 #include "gq_aux_kernels.cuh"
+#include "gq_gemm.cuh"
 #include "gq_kernels.cuh"
 #include "gq_rowquant_tma.cuh"
 
@@ -436,6 +439,35 @@ gq_status quantize_batch(const gq_tensor* t, int n, Op op, bool f16_mode, void* 
     return run_passthrough(pass, stream);
 }
 
+// ---------------------------------------------------- dequant-on-load GEMM --
+
+std::atomic<void*> g_encode_tiled{nullptr};
+std::atomic<int> g_gemm_smem_set[kMaxDevices];
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no
+// link-time dependency on the driver library).
+PFN_cuTensorMapEncodeTiled encode_tiled() {
+    void* f = g_encode_tiled.load(std::memory_order_acquire);
+    if (!f) {
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !f)
+            return nullptr;
+        g_encode_tiled.store(f, std::memory_order_release);
+    }
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled>(f);
+}
+
+// K splits: enough CTAs to cover the SMs twice for a small M, each split
+// keeping at least 8 K tiles, the count dividing the K tiles evenly.
+int gemm_splits(int64_t tiles_mn, int64_t k_tiles) {
+    const int64_t want = std::max<int64_t>(1, (2 * (int64_t)sm_count() + tiles_mn - 1) / tiles_mn);
+    int best = 1;
+    for (int64_t s = 1; s <= want && s <= k_tiles / 8; ++s)
+        if (k_tiles % s == 0) best = (int)s;
+    return best;
+}
+
 // Scratch of gq_export_pack_noalloc: a fixed device array that every call on
 // a device shares, for callers that cannot hand the library any device memory.
 constexpr size_t kNoAllocSlots = 64;                       // per-tensor groups per call
@@ -539,6 +571,65 @@ gq_status gq_dequant(const uint8_t* d_packed, const uint16_t* d_scale_f16, int q
     dequant_kernel<<<(unsigned)blocks, kBlockThreads, 0, stream>>>(
         d_packed, d_scale_f16, qbits, gran == GQ_PER_TENSOR, rows, cols, prb, d_out, out_dtype,
         vec_out, words);
+    return launch_status();
+}
+
+gq_status gq_gemm_dequant(const void* d_x, int64_t M, int64_t K, int64_t ldx, const uint8_t* d_packed,
+                          const uint16_t* d_scale_f16, int qbits, int64_t N, float* d_y, int64_t ldy,
+                          int32_t* d_status, cudaStream_t stream) {
+    if (M < 0 || N < 0 || K < 0 || (qbits != 6 && qbits != 8)) return GQ_ERR_INVALID_ARG;
+    if (ldx < K || ldy < N) return GQ_ERR_INVALID_ARG;
+    if (K % kGemmBK != 0 || M > INT32_MAX || K > INT32_MAX || N > INT32_MAX) return GQ_ERR_UNSUPPORTED;
+    if (d_status && !aligned(d_status, 4)) return GQ_ERR_MISALIGNED;
+    if (d_status && cuda_status(cudaMemsetAsync(d_status, 0, sizeof(int32_t), stream)) != GQ_OK) return GQ_ERR_CUDA;
+    if (M == 0 || N == 0) return GQ_OK;
+    if (!d_x || !d_packed || !d_scale_f16 || !d_y) return GQ_ERR_INVALID_ARG;
+    if (!aligned(d_x, 16) || (ldx % 8) != 0 || !aligned(d_packed, 16) || !aligned(d_scale_f16, 2) ||
+        !aligned(d_y, 16) || (ldy % 4) != 0)
+        return GQ_ERR_MISALIGNED;
+    if (K == 0)
+        return cuda_status(cudaMemset2DAsync(d_y, (size_t)ldy * 4, 0, (size_t)N * 4, (size_t)M, stream));
+    PFN_cuTensorMapEncodeTiled enc = encode_tiled();
+    if (!enc) return GQ_ERR_UNSUPPORTED;
+    GemmParams P;
+    std::memset(&P, 0, sizeof(P));
+    const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)M};
+    const cuuint64_t gstride[1] = {(cuuint64_t)ldx * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kGemmBK, (cuuint32_t)kGemmBM};
+    const cuuint32_t estride[2] = {1, 1};
+    if (enc(&P.tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(d_x), gdim, gstride, box, estride,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return GQ_ERR_UNSUPPORTED;
+    P.packed = d_packed;
+    P.scale = d_scale_f16;
+    P.y = d_y;
+    P.status = d_status;
+    P.M = M;
+    P.N = N;
+    P.K = K;
+    P.prb = packed_row_bytes(K, qbits);
+    P.ldy = ldy;
+    P.qbits = qbits;
+    const int64_t tiles_n = (N + kGemmBN - 1) / kGemmBN, tiles_m = (M + kGemmBM - 1) / kGemmBM;
+    if (tiles_n > 0x7FFFFFFF || tiles_m > 65535) return GQ_ERR_UNSUPPORTED;
+    const int64_t k_tiles = K / kGemmBK;
+    const int splits = gemm_splits(tiles_n * tiles_m, k_tiles);
+    P.k_tiles = (int32_t)(k_tiles / splits);
+    P.accumulate = splits > 1 ? 1 : 0;
+    if (splits > 1 &&
+        cuda_status(cudaMemset2DAsync(d_y, (size_t)ldy * 4, 0, (size_t)N * 4, (size_t)M, stream)) != GQ_OK)
+        return GQ_ERR_CUDA;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GQ_ERR_CUDA;
+    if (dev >= 0 && dev < kMaxDevices && g_gemm_smem_set[dev].load() < kGemmSmemBytes) {
+        if (cuda_status(cudaFuncSetAttribute(gemm_dequant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kGemmSmemBytes)) != GQ_OK)
+            return GQ_ERR_CUDA;
+        g_gemm_smem_set[dev].store(kGemmSmemBytes);
+    }
+    const dim3 grid((unsigned)tiles_n, (unsigned)tiles_m, (unsigned)splits);
+    gemm_dequant_kernel<<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(P);
     return launch_status();
 }
 

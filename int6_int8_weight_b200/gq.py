@@ -39,7 +39,7 @@ STATUS_NAMES = {0: "GQ_OK", 1: "GQ_ERR_INVALID_ARG", 2: "GQ_ERR_UNSUPPORTED",
                 6: "GQ_ERR_NONFINITE", 7: "GQ_ERR_CUDA", 8: "GQ_ERR_TIMEOUT"}
 
 EXPORTED = ("gq_row_clip_select", "gq_fakequant_fwd", "gq_fakequant_average", "gq_ste_bwd", "gq_export_pack",
-            "gq_export_pack_noalloc", "gq_dequant", "gq_workspace_size", "gq_packed_row_bytes", "gq_k_from_p",
+            "gq_export_pack_noalloc", "gq_dequant", "gq_gemm_dequant", "gq_workspace_size", "gq_packed_row_bytes", "gq_k_from_p",
             "gq_plan_kind", "gq_status_string", "gq_last_cuda_error", "gq_last_cuda_error_string")
 
 
@@ -79,9 +79,10 @@ def _load() -> C.CDLL:
     L.gq_export_pack_noalloc.argtypes = [T, i32, vp, vp]
     L.gq_ste_bwd.argtypes = [vp, vp, i32, i64, i32, vp]
     L.gq_dequant.argtypes = [vp, vp, i32, i32, i64, i64, vp, i32, vp]
+    L.gq_gemm_dequant.argtypes = [vp, i64, i64, i64, vp, vp, i32, i64, vp, i64, vp, vp]
     for f in ("gq_row_clip_select", "gq_fakequant_fwd", "gq_fakequant_average", "gq_export_pack",
               "gq_export_pack_noalloc",
-              "gq_ste_bwd", "gq_dequant"):
+              "gq_ste_bwd", "gq_dequant", "gq_gemm_dequant"):
         getattr(L, f).restype = i32
     L.gq_workspace_size.argtypes = [T, i32]
     L.gq_workspace_size.restype = sz
@@ -167,6 +168,11 @@ def gq_ste_bwd(g_out_ptr, g_w_ptr, dtype, numel, accumulate, stream=None):
 def gq_dequant(packed_ptr, scale_ptr, qbits, gran, rows, cols, out_ptr, out_dtype, stream=None):
     _check(LIB.gq_dequant(packed_ptr or None, scale_ptr or None, qbits, gran, rows, cols,
                           out_ptr or None, out_dtype, _stream(stream)), "gq_dequant")
+
+
+def gq_gemm_dequant(x_ptr, M, K, ldx, packed_ptr, scale_ptr, qbits, N, y_ptr, ldy, d_status=0, stream=None):
+    _check(LIB.gq_gemm_dequant(x_ptr, M, K, ldx, packed_ptr, scale_ptr, qbits, N, y_ptr, ldy,
+                               d_status or None, _stream(stream)), "gq_gemm_dequant")
 
 
 def gq_workspace_size(descs) -> int:
@@ -371,6 +377,23 @@ def dequant(packed: torch.Tensor, scale_f16: torch.Tensor, qbits: int, rows: int
                GQ_PER_TENSOR if per_tensor else GQ_PER_ROW, rows, cols, out.data_ptr(),
                _dtype_code(out), stream)
     return out
+
+
+def gemm_dequant(x: torch.Tensor, packed: torch.Tensor, scale_f16: torch.Tensor, qbits: int,
+                 y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Y = X @ W_hat^T with W_hat = bf16(q * s) rebuilt from the export's
+    packed codes and binary16 row scales inside the GEMM (tcgen05).  ``x``
+    is bf16 [M, K] (rows contiguous), ``packed`` uint8 [N, packed row bytes]
+    and ``scale_f16`` fp16 [N]; Y is fp32 [M, N]."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a bf16 [M, K] tensor with contiguous rows")
+    M, K = x.shape
+    N = packed.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    gq_gemm_dequant(x.data_ptr(), M, K, x.stride(0), packed.data_ptr(), scale_f16.data_ptr(), qbits, N,
+                    y.data_ptr(), y.stride(0), 0, stream)
+    return y
 
 
 def ste_bwd(g_out: torch.Tensor, g_w: torch.Tensor | None = None, stream=None) -> torch.Tensor:
