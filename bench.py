@@ -47,6 +47,7 @@ import synth  # noqa: E402
 METRIC = "weight GB/s through fused fake-quant+export and % of B200 HBM peak"
 UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 WORKLOAD = ("bandwidth stress: fp32 16384x16384, 65536x4096, 262144x512 and bf16 copies "
             "(Student-t nu=3, std 0.02); per matrix int6 per-row p=0.9999 clip-select+"
             "fake-quant+pack (w_hat, packed, fp16 scales) and int8 per-row absmax "
@@ -99,6 +100,16 @@ def job_throughput(units_per_rank: float, elapsed_s_per_rank: float, world: int,
 
 
 # ------------------------------------------------------------------ peaks --
+
+def bf16_peak():
+    """Dense bf16 tensor peak (TFLOP/s): the measured cuBLAS burst figure."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
 
 def hbm_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -307,11 +318,15 @@ def measure_rows(gq, device, peak):
             ts.append(s.elapsed_time(e) / 1e3)
         return statistics.median(ts)
 
-    def record(name, seconds, alg_bytes, in_bytes, launches, note=""):
+    def record(name, seconds, alg_bytes, in_bytes, launches, note="", flops=None):
         gbs = alg_bytes / seconds / 1e9
         out[name] = {"ms": round(seconds * 1e3, 4), "weight_gbs": round(in_bytes / seconds / 1e9, 1),
                      "alg_gbs": round(gbs, 1), "hbm_frac": round(gbs / peak, 3),
                      "launches": launches, **({"note": note} if note else {})}
+        if flops is not None:
+            tf = flops / seconds / 1e12
+            out[name]["tflops"] = round(tf, 1)
+            out[name]["tensor_frac"] = round(tf / tf_peak, 3)
 
     # STE backward on the 16384^2 shape: copy (fp32) and accumulate (bf16)
     n = 16384 * 16384
@@ -353,6 +368,29 @@ def measure_rows(gq, device, peak):
                timed(lambda: gq.LIB.gq_fakequant_average(arr0, aa, 1, 0, None, 0, None, None)),
                10 * n, 2 * n, 1, note="reads w (2 B) and the binary32 average (4 B), writes the average (4 B)")
     del W, o, outd, Wb, dqb, avg
+
+    # the consuming GEMM with the int6 dequant in its weight load (tcgen05),
+    # against cuBLAS on the pre-dequantized bf16 weight; decode-like (small M,
+    # weight-read bound) and prefill-like (tensor bound) shapes
+    tf_peak, _ = bf16_peak()
+    for M, N, K in ((16, 16384, 16384), (128, 16384, 16384), (4096, 8192, 8192)):
+        Wg = synth.draw_bandwidth_matrix(N, K, 0, device=device)
+        (q,) = gq.export_pack([gq.Request(Wg, 6, 0.9999, want_dq=False)], check_status=False)
+        del Wg
+        X = (torch.randn(M, K, device=device) * 0.5).to(torch.bfloat16)
+        Y = torch.empty(M, N, device=device)
+        wbytes = q.packed.numel() + 2 * N
+        alg = wbytes + 2 * M * K + 4 * M * N
+        fl = 2 * M * N * K
+        record(f"gemm dequant-on-load int6 M{M} N{N} K{K}",
+               timed(lambda: gq.gemm_dequant(X, q.packed, q.scale_f16, 6, y=Y), flush_between=True),
+               alg, wbytes, 1, note="packed int6 + fp16 scales + bf16 X read, fp32 Y written", flops=fl)
+        Wh = gq.dequant(q.packed, q.scale_f16, 6, N, K, out_dtype=torch.bfloat16)
+        record(f"cuBLAS bf16 on pre-dequantized weight M{M} N{N} K{K}",
+               timed(lambda: torch.matmul(X, Wh.t()), flush_between=True),
+               2 * N * K + 2 * M * K + 2 * M * N, 2 * N * K, None,
+               note="torch.matmul, bf16 W_hat read, bf16 Y; not counting the dequant pass", flops=fl)
+        del q, X, Y, Wh
 
     # model-shaped batched workloads (L2-resident: flushed between reps)
     def batch(specs_arrays, export=True, per_tensor_override=None, name="", note=""):

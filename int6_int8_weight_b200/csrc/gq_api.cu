@@ -458,13 +458,22 @@ PFN_cuTensorMapEncodeTiled encode_tiled() {
     return reinterpret_cast<PFN_cuTensorMapEncodeTiled>(f);
 }
 
-// K splits: enough CTAs to cover the SMs twice for a small M, each split
-// keeping at least 8 K tiles, the count dividing the K tiles evenly.
-int gemm_splits(int64_t tiles_mn, int64_t k_tiles) {
-    const int64_t want = std::max<int64_t>(1, (2 * (int64_t)sm_count() + tiles_mn - 1) / tiles_mn);
+// K splits for a grid of tiles_mn output tiles: the split count minimising
+// (waves of one-CTA-per-SM launches) x (per-CTA time), with a per-CTA cost
+// of about 5 us plus 0.15 us per 64-wide K stage (measured on the decode
+// shapes); each split keeps at least 8 stages.
+int gemm_splits(int64_t tiles_mn, int64_t k_stages) {
+    const double sms = (double)sm_count();
     int best = 1;
-    for (int64_t s = 1; s <= want && s <= k_tiles / 8; ++s)
-        if (k_tiles % s == 0) best = (int)s;
+    double best_t = 1e30;
+    for (int64_t s = 1; s <= std::max<int64_t>(1, k_stages / 8) && s <= 64; ++s) {
+        const double waves = std::ceil((double)(tiles_mn * s) / sms);
+        const double t = waves * (5.0 + 0.15 * std::ceil((double)k_stages / (double)s));
+        if (t < best_t - 1e-9) {
+            best_t = t;
+            best = (int)s;
+        }
+    }
     return best;
 }
 
@@ -593,30 +602,61 @@ gq_status gq_gemm_dequant(const void* d_x, int64_t M, int64_t K, int64_t ldx, co
     if (!enc) return GQ_ERR_UNSUPPORTED;
     GemmParams P;
     std::memset(&P, 0, sizeof(P));
+    // a batch of at most 128 tokens swaps the operands: 128 weight rows x nt tokens
+    P.swap = M <= kGemmBM ? 1 : 0;
+    P.nt = kGemmBM;
+    if (P.swap) {
+        P.nt = 16;
+        while (P.nt < M) P.nt *= 2;
+    }
+    P.idesc = gemm_idesc(kGemmBM, P.swap ? (uint32_t)P.nt : (uint32_t)kGemmBN);
+    P.acc_cols = P.swap ? (uint32_t)std::max(32, P.nt) : (uint32_t)kGemmBN;
+    P.tmem_cols = P.acc_cols * kGemmMmaWarps;
     const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)M};
     const cuuint64_t gstride[1] = {(cuuint64_t)ldx * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)kGemmBK, (cuuint32_t)kGemmBM};
+    const cuuint32_t box[2] = {(cuuint32_t)kGemmBK, (cuuint32_t)P.nt};
     const cuuint32_t estride[2] = {1, 1};
     if (enc(&P.tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(d_x), gdim, gstride, box, estride,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return GQ_ERR_UNSUPPORTED;
-    P.packed = d_packed;
+    const int64_t prb = packed_row_bytes(K, qbits);
+    const cuuint64_t wdim[2] = {(cuuint64_t)prb, (cuuint64_t)N};
+    const cuuint64_t wstride[1] = {(cuuint64_t)prb};
+    const int64_t stage_code_bytes = qbits == 6 ? 48 : 64;       // 64 codes of a row
+    const cuuint32_t wbox[2] = {(cuuint32_t)stage_code_bytes, (cuuint32_t)kGemmBN};
+    if (enc(&P.tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(d_packed), wdim, wstride, wbox,
+            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return GQ_ERR_UNSUPPORTED;
     P.scale = d_scale_f16;
     P.y = d_y;
     P.status = d_status;
     P.M = M;
     P.N = N;
     P.K = K;
-    P.prb = packed_row_bytes(K, qbits);
     P.ldy = ldy;
     P.qbits = qbits;
-    const int64_t tiles_n = (N + kGemmBN - 1) / kGemmBN, tiles_m = (M + kGemmBM - 1) / kGemmBM;
+    const int64_t tiles_n = (N + kGemmBN - 1) / kGemmBN, tiles_m = (M + P.nt - 1) / P.nt;
     if (tiles_n > 0x7FFFFFFF || tiles_m > 65535) return GQ_ERR_UNSUPPORTED;
-    const int64_t k_tiles = K / kGemmBK;
-    const int splits = gemm_splits(tiles_n * tiles_m, k_tiles);
-    P.k_tiles = (int32_t)(k_tiles / splits);
+    const int64_t k_stages = K / kGemmBK;
+    const int splits = gemm_splits(tiles_n * tiles_m, k_stages);
+    P.k_stages = (int32_t)k_stages;
+    P.splits = splits;
     P.accumulate = splits > 1 ? 1 : 0;
+    // ring depths, all even: a waiter then always has seen the barrier's
+    // previous phase itself (stages alternate between two MMA warps and two
+    // dequant groups), so a parity test cannot be satisfied by a phase
+    // behind the one it waits for
+    const int64_t x_bytes = (int64_t)P.nt * 128;
+    const int64_t code_bytes = kGemmBN * stage_code_bytes;
+    // (the X ring covers a round trip X load -> dequant check -> MMA ->
+    // commit -> next X load of about 2 us; small token tiles take it deep)
+    P.w_stages = P.nt == 128 ? 4 : 6;
+    P.x_stages = P.nt <= 32 ? 14 : 8;
+    P.c_stages = (int32_t)std::min<int64_t>(
+        kGemmCStagesMax, (kGemmRingBytes - P.w_stages * (int64_t)kGemmAtomBytes - P.x_stages * x_bytes) / code_bytes);
+    P.c_stages &= ~1;
     if (splits > 1 &&
         cuda_status(cudaMemset2DAsync(d_y, (size_t)ldy * 4, 0, (size_t)N * 4, (size_t)M, stream)) != GQ_OK)
         return GQ_ERR_CUDA;
