@@ -641,6 +641,36 @@ def run_reference(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_gemm(args):
+    """The dequant-on-load GEMM alone on one shape (``--gemm M,N,K,QBITS``):
+    synthetic weight exported through libgq, random bf16 X, ``warmup`` then
+    ``steps`` back-to-back calls timed with CUDA events.  An entry point for
+    profiling that kernel; it prints one JSON line of its own."""
+    import torch
+    from int6_int8_weight_b200 import gq
+    M, N, K, qbits = (int(v) for v in args.gemm.split(","))
+    device = torch.device("cuda")
+    W = synth.draw_bandwidth_matrix(N, K, 0, device=device)
+    (q,) = gq.export_pack([gq.Request(W, qbits, 0.9999, want_dq=False)], check_status=False)
+    del W
+    X = (torch.randn(M, K, device=device) * 0.5).to(torch.bfloat16)
+    Y = torch.empty(M, N, device=device)
+    for _ in range(args.warmup):
+        gq.gemm_dequant(X, q.packed, q.scale_f16, qbits, y=Y)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        gq.gemm_dequant(X, q.packed, q.scale_f16, qbits, y=Y)
+    b.record()
+    torch.cuda.synchronize()
+    us = a.elapsed_time(b) * 1e3 / max(args.steps, 1)
+    wbytes = q.packed.numel() + 2 * N
+    print(json.dumps({"gemm": f"M{M} N{N} K{K} int{qbits}", "us_per_call": round(us, 2),
+                      "tflops": round(2 * M * N * K / us / 1e6, 1),
+                      "alg_gbs": round((wbytes + 2 * M * K + 4 * M * N) / us / 1e3, 1)}), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -654,7 +684,12 @@ def main(argv=None):
     ap.add_argument("--only", default=None,
                     help="restrict the step to calls whose name contains this text, "
                          "underscores for spaces, e.g. f32_16384x16384_int6")
+    ap.add_argument("--gemm", default=None,
+                    help="profile the dequant-on-load GEMM alone on M,N,K,QBITS (one JSON line of its own)")
     args = ap.parse_args(argv)
+    if args.gemm:
+        run_gemm(args)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     world, rank, local = dist_env()
