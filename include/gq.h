@@ -284,8 +284,14 @@ GQ_API gq_status gq_dequant(const uint8_t* d_packed, const uint16_t* d_scale_f16
  * the bf16 fake-quant weight the forward pass would multiply by; it is
  * rebuilt tile by tile in shared memory and never written to memory.
  *   d_x      bf16 [M, ldx] activations, row-major, 16-byte aligned, ldx % 8 == 0
+ *   d_packed [N, gq_packed_row_bytes(K, qbits)] bytes, 16-byte aligned
+ *   d_scale_f16 [N] binary16 bit patterns, 2-byte aligned
  *   d_y      fp32 [M, ldy] output, overwritten; 16-byte aligned, ldy % 4 == 0
- *   d_status nullable: GQ_STATUS_TIMEOUT if a bounded wait on the device gave up
+ *   d_status nullable: set to 0 on the stream, then GQ_STATUS_TIMEOUT if a
+ *            bounded wait on the device gave up (Y is then not valid)
+ * All buffers are the caller's; the call allocates nothing, checks its
+ * arguments on the host before launching, and runs asynchronously on
+ * `stream` (one kernel launch, plus a memset of Y when K is split).
  * Products are exact (bf16 x bf16) and accumulate in binary32 in the tensor
  * cores' order, so Y is not bitwise reproducible against a sequential sum:
  * |Y - exact| <= (K/8 + 4) * 2^-24 * sum_k |X[m, k] * W_hat[n, k]|.
