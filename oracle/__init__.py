@@ -68,6 +68,8 @@ class Oracle:
         L.or_dequant.restype = i32
         L.or_ste_bwd.argtypes = [vp, vp, i32, i64, i32]
         L.or_ste_bwd.restype = i32
+        L.or_col_scale.argtypes = [vp, i32, i64, i64, i64, vp, vp]
+        L.or_col_scale.restype = i32
         L.or_passthrough_f16.argtypes = [vp, i32, i64, vp]
         L.or_passthrough_f16.restype = i32
         L.or_average_update.argtypes = [vp, vp, i32, i64, i32, i64, f32]
@@ -93,14 +95,35 @@ class Oracle:
     def packed_row_bytes(self, cols: int, qbits: int) -> int:
         return int(self.L.or_packed_row_bytes(cols, qbits))
 
+    def col_scale(self, w: np.ndarray, t: np.ndarray, cols: int | None = None) -> np.ndarray:
+        """AWQ column scaling (reading R12 in gq_oracle.c): the dense
+        [rows, cols] weight RN_dtype(w[r, c] * t[c]) in w's dtype."""
+        assert w.ndim == 2
+        w = np.ascontiguousarray(w)
+        rows, ld = w.shape
+        cols = ld if cols is None else cols
+        t = np.ascontiguousarray(t, dtype=np.float32).ravel()
+        assert t.size >= cols
+        out = np.zeros((rows, cols), w.dtype)
+        st = self.L.or_col_scale(_ptr(w), _dtype_code(w), rows, cols, ld, _ptr(t), _ptr(out))
+        if st != OR_OK:
+            raise ValueError(f"oracle col_scale status {st}")
+        return out
+
     def quantize(self, w: np.ndarray, qbits: int, p: float = 1.0,
                  per_tensor: bool = False, export: bool = True,
-                 cols: int | None = None) -> QuantResult:
+                 cols: int | None = None, col_scale: np.ndarray | None = None) -> QuantResult:
         """Fake-quant forward / export of a 2-D weight ``w`` ([rows, ld]).
 
         ``cols`` (default: all of ``ld``) selects the used columns of each row.
+        ``col_scale`` (AWQ, per-row only): quantize RN_dtype(w * t[column])
+        instead of w.
         """
         assert w.ndim == 2
+        if col_scale is not None:
+            assert not per_tensor, "column scaling is defined for per-row groups"
+            w = self.col_scale(w, col_scale, cols)
+            cols = None
         w = np.ascontiguousarray(w)
         rows, ld = w.shape
         cols = ld if cols is None else cols

@@ -25,7 +25,8 @@
  *    "Quantization" (int8, bits 8, scope embeddings).
  *  - "Add non-record submission: 12L 24min Vocab1792 ... Int6AWQ MixedBits"
  *    (PR #1495), "Mixed-bit quantization details" (int6 default, named
- *    tensors promoted to int8).
+ *    tensors promoted to int8); the summary list and the Community Review
+ *    (AWQ column scaling from activation statistics).
  *
  * The pages give bit widths, the int6 range and the list of features, but no
  * rounding rule, percentile definition, scale format or packing layout.  The
@@ -63,6 +64,16 @@
  *   R11 exponential moving average of the snapshots: a' = d*a + c*x with
  *      c = 1 - d, each product, the difference and the sum one binary32
  *      operation (the pages give d = 0.997).
+ *   R12 AWQ column scaling ("... Int6AWQ MixedBits", PR #1495: "mixed-bit
+ *      int6 AWQ" export, and its Community Review: activation statistics
+ *      collected for "AWQ column scaling" before post-training
+ *      quantization).  The pages give no rule from the statistics to the
+ *      scales, so the per-column scale vector t[cols] (binary32) is an
+ *      input.  The weight is rescaled column by column in its own dtype,
+ *      w'[r, c] = RN_dtype(w[r, c] * t[c]) (the product one binary32
+ *      multiply; bf16 then rounded to nearest even), and w' goes through the
+ *      unchanged per-row clip, scale, quantize, dequant and pack.  The
+ *      activations are divided by t at inference, outside the quantizer.
  *
  * Build: plain C11, gcc -O2 -ffp-contract=off, no fast-math, SSE (never x87)
  * binary32 arithmetic, default rounding mode (round to nearest even).
@@ -488,6 +499,28 @@ int or_average_update(float* a, const void* x, int dtype, int64_t numel, int kin
         return OR_OK;
     }
     return OR_ERR_ARG;
+}
+
+/*
+ * AWQ column scaling (R12): out[r, c] = RN_dtype(w[r, ld-strided] * t[c]),
+ * dense [rows, cols] in the input dtype.  The result is the weight that the
+ * per-row quantizer (or_quantize) then takes.
+ */
+int or_col_scale(const void* w, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                 const float* t, void* out)
+{
+    if (!w || !t || !out || rows < 0 || cols < 0 || ld < cols)
+        return OR_ERR_ARG;
+    if (dtype != OR_F32 && dtype != OR_BF16)
+        return OR_ERR_ARG;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t c = 0; c < cols; ++c) {
+            float x = load_elem(w, dtype, r * ld + c);
+            float y = x * t[c];                    /* one binary32 multiply */
+            store_elem(out, dtype, r * cols + c, y);
+        }
+    }
+    return OR_OK;
 }
 
 /* Small-tensor passthrough: binary16 round-to-nearest-even of each value. */

@@ -45,6 +45,12 @@ MUTANTS = {
     "mean_drops_average": ("a[i] = a[i] + u;", "a[i] = u;"),
     "ema_wrong_factor": ("float added = c * xi;", "float added = decay * xi;"),
     "ema_sign": ("float c = 1.0f - decay;", "float c = decay - 1.0f;"),
+    "colscale_divides": ("float y = x * t[c];", "float y = x / t[c];"),
+    "colscale_first_entry": ("float y = x * t[c];", "float y = x * t[0];"),
+    "colscale_dense_read": ("float x = load_elem(w, dtype, r * ld + c);",
+                            "float x = load_elem(w, dtype, r * cols + c);"),
+    "colscale_drops_last": ("for (int64_t c = 0; c < cols; ++c) {\n            float x = load_elem(w, dtype, r * ld + c);",
+                            "for (int64_t c = 0; c + 1 < cols; ++c) {\n            float x = load_elem(w, dtype, r * ld + c);"),
 }
 
 CHECKS = [   # cheapest first: a mutant stops at the first pin that rejects it
@@ -60,6 +66,7 @@ CHECKS = [   # cheapest first: a mutant stops at the first pin that rejects it
     pins.check_invariants,
     pins.check_pack_roundtrip_exhaustive,
     pins.check_average,
+    pins.check_col_scale,
 ]
 
 

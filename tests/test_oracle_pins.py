@@ -10,7 +10,10 @@
 * snapshot averaging: the first snapshot is copied, and the mean of two
   snapshots, a mean step with weight 1/4 and an EMA step with decay 1/2
   equal the exact rational results on dyadic inputs; decay 0 / 1 keep the
-  snapshot / the average; a long EMA of a constant follows 1 - d^k.
+  snapshot / the average; a long EMA of a constant follows 1 - d^k,
+* AWQ column scaling: every element equals the exact rational product rounded
+  once to binary32 (and to bf16 for bf16 weights); t = 1 and a uniform power
+  of two leave the codes unchanged.
 
 The ``orc`` fixture is parametrised so that ``test_oracle_mutants.py`` can run
 the same checks against oracle copies with a planted mistake.
@@ -556,3 +559,46 @@ def test_fakequant_average_composes(orc):
     ref, a = orc.fakequant_average(w, avg, 6, 0.99, oracle.AVG_MEAN, count=2)
     assert np.array_equal(a, orc.average_update(avg, ref.dq, oracle.AVG_MEAN, count=2))
     assert np.array_equal(ref.dq, orc.quantize(w, 6, 0.99, export=False).dq)
+
+
+def check_col_scale(orc, seed=41):
+    """AWQ column scaling (reading R12): each element is the exact product
+    w[r, c] * t[c] rounded once to binary32 (then, for bf16 weights, to the
+    nearest even bf16), computed here with rational arithmetic; t = 1 leaves
+    the weight and its quantization unchanged; a uniform power of two scales
+    the codes' clip and scale exactly."""
+    rng = np.random.default_rng(seed)
+    rows, cols, ld = 5, 37, 41                       # rows != cols, strided rows
+    w = np.zeros((rows, ld), np.float32)
+    w[:, :cols] = (rng.standard_normal((rows, cols)) * 0.03).astype(np.float32)
+    w[:, cols:] = 1e30                               # past the used columns: never read
+    t = (rng.random(cols) * 3.0 + 0.05).astype(np.float32)
+    got = orc.col_scale(w, t, cols)
+    for r in range(rows):
+        for c in range(cols):
+            want = exact.rn32(Fraction(float(w[r, c])) * Fraction(float(t[c])))
+            assert Fraction(float(got[r, c])) == want, (r, c)
+    wb = synth.to_bf16_bits(w[:, :cols]).reshape(rows, cols)
+    gotb = orc.col_scale(wb, t)
+    for r in range(rows):
+        for c in range(cols):
+            x = Fraction(float((np.uint32(wb[r, c]) << np.uint32(16)).view(np.float32)))
+            want = exact.rnbf16(exact.rn32(x * Fraction(float(t[c]))))
+            have = Fraction(float((np.uint32(gotb[r, c]) << np.uint32(16)).view(np.float32)))
+            assert have == want, (r, c)
+    # t = 1: the same weight, the same export
+    ones = np.ones(cols, np.float32)
+    assert np.array_equal(orc.col_scale(w, ones, cols).view(np.uint32), w[:, :cols].view(np.uint32))
+    a = orc.quantize(w[:, :cols].copy(), 6, 0.95, col_scale=ones)
+    b = orc.quantize(w[:, :cols].copy(), 6, 0.95)
+    assert np.array_equal(a.packed, b.packed) and np.array_equal(a.scale_f16, b.scale_f16)
+    # a uniform power of two: the same codes, clip and scale times 4 (training mode)
+    four = np.full(cols, 4.0, np.float32)
+    a = orc.quantize(w[:, :cols].copy(), 8, 0.9, export=False, col_scale=four)
+    b = orc.quantize(w[:, :cols].copy(), 8, 0.9, export=False)
+    assert np.array_equal(a.codes, b.codes)
+    assert np.array_equal(a.clip, b.clip * 4) and np.array_equal(a.scale_f32, b.scale_f32 * 4)
+
+
+def test_col_scale_pins(orc):
+    check_col_scale(orc)
