@@ -367,7 +367,20 @@ def measure_rows(gq, device, peak):
         record(f"fakequant + snapshot {name} bf16 16384^2 int6 (average only)",
                timed(lambda: gq.LIB.gq_fakequant_average(arr0, aa, 1, 0, None, 0, None, None)),
                10 * n, 2 * n, 1, note="reads w (2 B) and the binary32 average (4 B), writes the average (4 B)")
-    del W, o, outd, Wb, dqb, avg
+    # AWQ: int6 per-row export of the column-scaled bf16 weight (w_hat,
+    # packed codes, fp16 scales), column scales from synthetic statistics
+    t_awq = torch.from_numpy(synth.awq_col_scales(np.random.default_rng(3), 16384)).to(device)
+    pk = torch.empty(16384, gq.gq_packed_row_bytes(16384, 6), dtype=torch.uint8, device=device)
+    h16 = torch.empty(16384, dtype=torch.float16, device=device)
+    da = gq.GQTensor(w=Wb.data_ptr(), dtype=1, qbits=6, gran=0, reserved=0, rows=16384, cols=16384,
+                     ld=16384, p=0.9999, dq=dqb.data_ptr(), codes=0, packed=pk.data_ptr(),
+                     scale_f16=h16.data_ptr(), scale_f32=0, clip=0, col_scale=t_awq.data_ptr())
+    arra = gq._arr([da])
+    record("AWQ column-scaled export bf16 16384^2 int6 p=0.9999",
+           timed(lambda: gq.LIB.gq_export_pack(arra, 1, None, 0, None, None)),
+           4.75 * n + 2 * 16384 + 4 * 16384, 2 * n, 1,
+           note="reads w (2 B), writes w_hat (2 B) + packed (0.75 B); row kernel (reads the row twice)")
+    del W, o, outd, Wb, dqb, avg, pk, h16, t_awq
 
     # the consuming GEMM with the int6 dequant in its weight load (tcgen05),
     # against cuBLAS on the pre-dequantized bf16 weight; decode-like (small M,

@@ -149,6 +149,19 @@ typedef struct gq_tensor {
     uint16_t* scale_f16;
     float* scale_f32;
     float* clip;
+    /* AWQ column scaling, nullable: binary32 [cols] per-column scales t.
+     * When given, the group quantized is the column-scaled weight
+     * w'[r, c] = RN_dtype(w[r, c] * t[c]) (one binary32 multiply; a bf16
+     * weight is then rounded to nearest even bf16), and clip, scales, codes,
+     * packed and dq are those of w'.  Per-row groups of gq_row_clip_select,
+     * gq_fakequant_fwd, gq_fakequant_average and gq_export_pack only
+     * (GQ_ERR_UNSUPPORTED with GQ_PER_TENSOR or qbits 16); 4-byte aligned.
+     * The pages give no rule from activation statistics to t, so t is the
+     * caller's; the activations are divided by t at inference.  Source:
+     * "... Int6AWQ MixedBits" (PR #1495): "mixed-bit int6 AWQ" export and,
+     * in its Community Review, activation statistics collected for AWQ
+     * column scaling before post-training quantization. */
+    const float* col_scale;
 } gq_tensor;
 
 /*

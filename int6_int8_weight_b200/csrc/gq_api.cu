@@ -6,6 +6,7 @@
 #include <algorithm>
 #include <atomic>
 #include <cmath>
+#include <cstddef>
 #include <cstring>
 #include <string>
 #include <vector>
@@ -71,6 +72,9 @@ gq_status check_avg(const gq_tensor& t, const gq_avg& a) {
     return GQ_OK;
 }
 
+static_assert(sizeof(gq_tensor) == 112 && offsetof(gq_tensor, col_scale) == 104,
+              "gq_tensor layout is part of the ABI (the Python binding mirrors it)");
+
 gq_status check_tensor(const gq_tensor& t, Op op, bool f16_mode) {
     if (t.reserved != 0) return GQ_ERR_INVALID_ARG;
     if (t.dtype != GQ_F32 && t.dtype != GQ_BF16) return GQ_ERR_INVALID_ARG;
@@ -80,6 +84,8 @@ gq_status check_tensor(const gq_tensor& t, Op op, bool f16_mode) {
     if (t.rows < 0 || t.cols < 0 || t.ld < t.cols) return GQ_ERR_INVALID_ARG;
     if (t.cols > (int64_t)INT32_MAX) return GQ_ERR_UNSUPPORTED;
     if (!pass16 && !(t.p > 0.0 && t.p <= 1.0)) return GQ_ERR_INVALID_ARG;
+    // AWQ column scales: per-row groups of the quantizing calls only
+    if (t.col_scale && (pass16 || t.gran != GQ_PER_ROW)) return GQ_ERR_UNSUPPORTED;
     const int64_t esz = t.dtype == GQ_F32 ? 4 : 2;
     if (t.rows > 0 && t.ld > 0 && t.rows > INT64_MAX / 16 / t.ld) return GQ_ERR_INVALID_ARG;
     if (t.rows > 0 && t.cols > 0 && t.rows > INT64_MAX / 16 / t.cols) return GQ_ERR_INVALID_ARG;
@@ -90,6 +96,7 @@ gq_status check_tensor(const gq_tensor& t, Op op, bool f16_mode) {
     if (t.scale_f16 && !aligned(t.scale_f16, 2)) return GQ_ERR_MISALIGNED;
     if (t.scale_f32 && !aligned(t.scale_f32, 4)) return GQ_ERR_MISALIGNED;
     if (t.clip && !aligned(t.clip, 4)) return GQ_ERR_MISALIGNED;
+    if (t.col_scale && !aligned(t.col_scale, 4)) return GQ_ERR_MISALIGNED;
     switch (op) {
         case Op::Select:
             if (!t.clip) return GQ_ERR_INVALID_ARG;
@@ -386,8 +393,10 @@ gq_status quantize_batch(const gq_tensor* t, int n, Op op, bool f16_mode, void* 
                 D.avg_c = 1.0f - A.decay;                   // one binary32 subtraction
             }
         }
+        D.colscale = T.col_scale;
         const bool elem = T.dq || T.codes || T.packed || D.avg;
         int32_t flags = elem ? kElemOut : 0;
+        if (T.col_scale && aligned(T.col_scale, 16)) flags |= kVecCol;
         if (D.avg && aligned(D.avg, 16) && (T.cols % 4) == 0) flags |= kVecAvg;
         const size_t vin = T.dtype == GQ_F32 ? 16 : 8;
         if (aligned(T.w, vin) && ((T.ld * esz) % (int64_t)vin) == 0) flags |= kVecIn;
@@ -420,7 +429,7 @@ gq_status quantize_batch(const gq_tensor* t, int n, Op op, bool f16_mode, void* 
             D.items = T.rows;
         }
         D.flags = flags;
-        if (tma_eligible(T, flags))
+        if (tma_eligible(T, flags) && !T.col_scale)   // column-scaled rows: the row kernels
             rows_tma.push_back(D);
         else if (T.cols <= 2048)
             rows_w.push_back(D);

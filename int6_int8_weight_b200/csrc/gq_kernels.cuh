@@ -45,6 +45,7 @@ struct RowDesc {
     float* avg;                // binary32 [rows, cols] averages (dense), or null
     float avg_t;               // mean: RN(1 / (n + 1)); EMA: decay
     float avg_c;               // EMA: RN(1 - decay)
+    const float* colscale;     // AWQ: binary32 [cols] column scales, or null
 };
 
 constexpr int32_t kVecIn = 1;       // rows of w are 16-byte (f32) / 8-byte (bf16) aligned
@@ -54,6 +55,7 @@ constexpr int32_t kVecPacked = 8;   // rows of packed 4-byte aligned
 constexpr int32_t kPerTensor = 16;
 constexpr int32_t kElemOut = 32;    // dq, codes, packed or an average requested
 constexpr int32_t kVecAvg = 64;     // rows of the average 16-byte aligned
+constexpr int32_t kVecCol = 128;    // the column scales 16-byte aligned
 
 struct RowParams {
     int32_t ndesc;
@@ -71,9 +73,18 @@ __device__ __forceinline__ int find_desc(const int64_t* start, int n, int64_t it
     return lo;
 }
 
-// Four consecutive elements of a row (elements past n read as 0).
+// Four consecutive elements of a row (elements past n read as 0).  With
+// column scales cs (AWQ), element e is the column-scaled weight
+// RN_dtype(w[e] * cs[e]): one binary32 multiply, rounded to nearest even
+// bf16 for a bf16 weight (the weight rescaled in its own dtype).
+__device__ __forceinline__ float col_scaled(float x, float t, int dtype) {
+    const float y = __fmul_rn(x, t);
+    return dtype == kF32 ? y : bf16_bits_to_float(float_to_bf16_bits(y));
+}
+
 __device__ __forceinline__ void load_quad(const char* rowp, int dtype, int64_t e0, int64_t n,
-                                          bool vec, float v[4]) {
+                                          bool vec, float v[4], const float* cs = nullptr,
+                                          bool vcs = false) {
     if (vec && e0 + 3 < n) {
         if (dtype == kF32) {
             float4 x = *reinterpret_cast<const float4*>(rowp + e0 * 4);
@@ -85,19 +96,32 @@ __device__ __forceinline__ void load_quad(const char* rowp, int dtype, int64_t e
             v[2] = bf16_bits_to_float(x.y & 0xFFFFu);
             v[3] = bf16_bits_to_float(x.y >> 16);
         }
-        return;
-    }
+    } else {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        int64_t e = e0 + i;
-        float x = 0.0f;
-        if (e < n) {
-            if (dtype == kF32)
-                x = reinterpret_cast<const float*>(rowp)[e];
-            else
-                x = bf16_bits_to_float(reinterpret_cast<const uint16_t*>(rowp)[e]);
+        for (int i = 0; i < 4; ++i) {
+            int64_t e = e0 + i;
+            float x = 0.0f;
+            if (e < n) {
+                if (dtype == kF32)
+                    x = reinterpret_cast<const float*>(rowp)[e];
+                else
+                    x = bf16_bits_to_float(reinterpret_cast<const uint16_t*>(rowp)[e]);
+            }
+            v[i] = x;
         }
-        v[i] = x;
+    }
+    if (cs) {
+        if (vcs && e0 + 3 < n) {
+            const float4 t = __ldg(reinterpret_cast<const float4*>(cs + e0));
+            v[0] = col_scaled(v[0], t.x, dtype);
+            v[1] = col_scaled(v[1], t.y, dtype);
+            v[2] = col_scaled(v[2], t.z, dtype);
+            v[3] = col_scaled(v[3], t.w, dtype);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                if (e0 + i < n) v[i] = col_scaled(v[i], __ldg(cs + e0 + i), dtype);
+        }
     }
 }
 
@@ -108,7 +132,7 @@ __device__ __forceinline__ void load_quad(const char* rowp, int dtype, int64_t e
 template <int TW, int M>
 __device__ uint2 select_topm(const char* rowp, int dtype, int64_t n, bool vec, int m,
                                 int tw_warp, int lane, int team,
-                                uint32_t (*s_lists)[kTopMax]) {
+                                uint32_t (*s_lists)[kTopMax], const float* cs, bool vcs) {
     TopM<M> T;
     T.init();
     const int64_t nq = (n + 3) >> 2;
@@ -116,7 +140,7 @@ __device__ uint2 select_topm(const char* rowp, int dtype, int64_t n, bool vec, i
         int64_t j = jb + lane;
         if (j < nq) {
             float v[4];
-            load_quad(rowp, dtype, 4 * j, n, vec, v);
+            load_quad(rowp, dtype, 4 * j, n, vec, v, cs, vcs);
 #pragma unroll
             for (int i = 0; i < 4; ++i) T.insert(abs_key(v[i]));
         }
@@ -145,7 +169,7 @@ __device__ uint2 select_topm(const char* rowp, int dtype, int64_t n, bool vec, i
 template <int TW>
 __device__ uint32_t select_radix(const char* rowp, int dtype, int64_t n, bool vec, int64_t m,
                                  int tw_warp, int lane, int team, uint32_t* hist,
-                                 uint32_t* bcast, bool* nonfinite) {
+                                 uint32_t* bcast, bool* nonfinite, const float* cs, bool vcs) {
     const int tt = tw_warp * 32 + lane;
     const int64_t nq = (n + 3) >> 2;
     uint32_t prefix = 0, pmask = 0;
@@ -161,7 +185,7 @@ __device__ uint32_t select_radix(const char* rowp, int dtype, int64_t n, bool ve
             int64_t j = jb + lane;
             if (j < nq) {
                 float v[4];
-                load_quad(rowp, dtype, 4 * j, n, vec, v);
+                load_quad(rowp, dtype, 4 * j, n, vec, v, cs, vcs);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     uint32_t key = abs_key(v[i]);
@@ -232,7 +256,7 @@ __device__ void quantize_row(const RowDesc& D, int64_t r, const Scale& S, int tw
         const int64_t e0 = 4 * j;
         const bool full = e0 + 3 < n;
         float v[4] = {0.f, 0.f, 0.f, 0.f};
-        if (valid) load_quad(rowp, D.dtype, e0, n, vin, v);
+        if (valid) load_quad(rowp, D.dtype, e0, n, vin, v, D.colscale, (D.flags & kVecCol) != 0);
         float b[4];
         int q[4];
 #pragma unroll
@@ -342,6 +366,8 @@ rowquant_kernel(const __grid_constant__ RowParams P) {
         const int esz = D.dtype == kF32 ? 4 : 2;
         const char* rowp = reinterpret_cast<const char*>(D.w) + r * D.ld * esz;
         const bool vin = D.flags & kVecIn;
+        const float* cs = D.colscale;
+        const bool vcs = (D.flags & kVecCol) != 0;
 
         uint32_t ckey;
         bool nonfinite = false;
@@ -351,16 +377,16 @@ rowquant_kernel(const __grid_constant__ RowParams P) {
             const int m = D.m;
             uint2 sel;
             if (m <= 1)
-                sel = select_topm<TW, 1>(rowp, D.dtype, D.cols, vin, 1, tw_warp, lane, team, s_lists);
+                sel = select_topm<TW, 1>(rowp, D.dtype, D.cols, vin, 1, tw_warp, lane, team, s_lists, cs, vcs);
             else if (m <= 2)
-                sel = select_topm<TW, 2>(rowp, D.dtype, D.cols, vin, m, tw_warp, lane, team, s_lists);
+                sel = select_topm<TW, 2>(rowp, D.dtype, D.cols, vin, m, tw_warp, lane, team, s_lists, cs, vcs);
             else if (m <= 4)
-                sel = select_topm<TW, 4>(rowp, D.dtype, D.cols, vin, m, tw_warp, lane, team, s_lists);
+                sel = select_topm<TW, 4>(rowp, D.dtype, D.cols, vin, m, tw_warp, lane, team, s_lists, cs, vcs);
             else if (m <= kTopMax)
-                sel = select_topm<TW, 8>(rowp, D.dtype, D.cols, vin, m, tw_warp, lane, team, s_lists);
+                sel = select_topm<TW, 8>(rowp, D.dtype, D.cols, vin, m, tw_warp, lane, team, s_lists, cs, vcs);
             else
                 sel.x = select_radix<TW>(rowp, D.dtype, D.cols, vin, m, tw_warp, lane, team,
-                                         s_hist[team], s_bcast[team], &nonfinite);
+                                         s_hist[team], s_bcast[team], &nonfinite, cs, vcs);
             ckey = sel.x;
             if (m <= kTopMax) nonfinite = sel.y >= 0x7F800000u;
         }

@@ -57,6 +57,7 @@ class GQTensor(C.Structure):
         ("p", C.c_double),
         ("dq", C.c_void_p), ("codes", C.c_void_p), ("packed", C.c_void_p),
         ("scale_f16", C.c_void_p), ("scale_f32", C.c_void_p), ("clip", C.c_void_p),
+        ("col_scale", C.c_void_p),
     ]
 
 
@@ -238,6 +239,7 @@ class Request:
     want_scale_f32: bool = False
     want_clip: bool = False
     cols: int | None = None
+    col_scale: torch.Tensor | None = None   # AWQ: fp32 [cols] column scales (per-row groups)
 
 
 def _as_2d(w: torch.Tensor):
@@ -278,6 +280,12 @@ def _prepare(reqs, export: bool):
                      rows=rows, cols=cols, ld=ld, p=float(r.p), dq=_ptr(o.dq),
                      codes=_ptr(o.codes), packed=_ptr(o.packed), scale_f16=_ptr(o.scale_f16),
                      scale_f32=_ptr(o.scale_f32), clip=_ptr(o.clip))
+        if r.col_scale is not None:
+            cs = r.col_scale
+            if cs.dtype != torch.float32 or cs.dim() != 1 or cs.stride(0) != 1 or cs.numel() < cols \
+                    or cs.device != dev:
+                raise ValueError("col_scale must be a contiguous fp32 [cols] tensor on the weight's device")
+            d.col_scale = cs.data_ptr()
         descs.append(d)
         outs.append(o)
     return descs, outs

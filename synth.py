@@ -15,6 +15,12 @@ copies are the round-to-nearest-even of the fp32 values):
   (the textbook construction), times ``std / sqrt(3)``.
 * ``outlier_mix``: ``z`` standard normal, ``u`` uniform [0, 1);
   ``0.2 z`` where ``u < 0.01`` else ``0.02 z``.
+* ``awq_col_scales(cols)``: per-input-column activation statistics
+  ``a = |z0| * exp(1.5 z1)`` (a few channels far louder than the rest), and
+  the column scales a quantizer takes from them in the AWQ style,
+  ``t = a^0.5 / sqrt(max(a^0.5) * min(a^0.5))`` in float64, rounded to fp32.
+  The pages give no rule from statistics to scales; this only draws an input
+  of the right kind.
 
 Host workloads use ``numpy.random.default_rng(seed)`` with tensors drawn in the
 manifest order below; the bandwidth workload is drawn on the GPU from a seeded
@@ -242,3 +248,11 @@ def random_matrix(rng, rows, cols, kind="normal"):
     else:
         raise ValueError(kind)
     return x.reshape(rows, cols)
+
+
+def awq_col_scales(rng, cols):
+    """fp32 [cols] column scales drawn from synthetic activation statistics
+    (recipe in the module docstring)."""
+    a = np.abs(rng.standard_normal(cols)) * np.exp(1.5 * rng.standard_normal(cols)) + 1e-3
+    r = np.sqrt(a)
+    return (r / math.sqrt(r.max() * r.min())).astype(np.float32)

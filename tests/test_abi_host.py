@@ -62,8 +62,9 @@ def test_header_compiles_as_c():
 
 
 def test_struct_layout_matches_binding(gq):
-    assert C.sizeof(gq.GQTensor) == 104
+    assert C.sizeof(gq.GQTensor) == 112      # static_assert(sizeof(gq_tensor) == 112) in gq_api.cu
     assert gq.GQTensor.p.offset == 48 and gq.GQTensor.clip.offset == 96
+    assert gq.GQTensor.col_scale.offset == 104
 
 
 def test_k_from_p_matches_oracle(gq):
@@ -158,6 +159,11 @@ def test_other_argument_errors(gq):
     assert L.gq_dequant(None, None, 6, 0, 0, 4, None, 0, None) == 0  # empty is a no-op
     # empty batch is a no-op
     assert L.gq_export_pack(gq._arr([]), 0, None, 0, None, None) == 0
+    # AWQ column scales: per-row quantizing groups only, 4-byte aligned
+    assert L.gq_export_pack(gq._arr([_desc(gq, col_scale=0x50002)]), 1, None, 0, None, None) == 3
+    assert L.gq_export_pack(gq._arr([_desc(gq, gran=1, col_scale=0x50000)]), 1, None, 0, None, None) == 2
+    assert L.gq_export_pack(gq._arr([_desc(gq, qbits=16, dq=0, scale_f16=0, col_scale=0x50000)]), 1, None, 0,
+                            None, None) == 2
 
 
 def test_last_cuda_error_starts_clear(gq):
