@@ -196,7 +196,7 @@ gq_status run_rows(const std::vector<RowDesc>& rows, cudaStream_t stream) {
 // Pipelined launch over the descriptors whose rows can be bulk-copied.
 constexpr int kTmaStageBytes = 68 * 1024;
 constexpr int kTmaMaxRowBytes = 96 * 1024;
-std::atomic<int> g_tma_smem_set[kMaxDevices];
+std::atomic<int> g_tma_smem_set[2][kMaxDevices];
 
 bool tma_eligible(const gq_tensor& T, int32_t flags) {
     const int64_t esz = T.dtype == GQ_F32 ? 4 : 2;
@@ -244,7 +244,8 @@ int32_t tma_out_mode(const RowDesc& D) {
     }
 }
 
-gq_status run_rows_tma(std::vector<RowDesc>& rows, cudaStream_t stream) {
+template <bool kColScale>
+gq_status run_rows_tma_impl(std::vector<RowDesc>& rows, cudaStream_t stream) {
     if (rows.empty()) return GQ_OK;
     int64_t max_row = 0;
     for (const RowDesc& D : rows) max_row = std::max<int64_t>(max_row, D.cols * (D.dtype == kF32 ? 4 : 2));
@@ -270,11 +271,12 @@ gq_status run_rows_tma(std::vector<RowDesc>& rows, cudaStream_t stream) {
     const size_t smem = (size_t)nstages * sb + kTmaExtraBytes;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return GQ_ERR_CUDA;
-    if (dev >= 0 && dev < kMaxDevices && g_tma_smem_set[dev].load() < (int)smem) {
-        if (cuda_status(cudaFuncSetAttribute(rowquant_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem)) != GQ_OK)
+    std::atomic<int>& smem_set = g_tma_smem_set[kColScale ? 1 : 0][dev >= 0 && dev < kMaxDevices ? dev : 0];
+    if (dev >= 0 && dev < kMaxDevices && smem_set.load() < (int)smem) {
+        if (cuda_status(cudaFuncSetAttribute(rowquant_tma_kernel<kColScale>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != GQ_OK)
             return GQ_ERR_CUDA;
-        g_tma_smem_set[dev].store((int)smem);
+        smem_set.store((int)smem);
     }
     for (size_t base = 0; base < rows.size(); base += kMaxDesc) {
         TmaParams P;
@@ -293,10 +295,19 @@ gq_status run_rows_tma(std::vector<RowDesc>& rows, cudaStream_t stream) {
         P.start[nd] = acc;
         if (acc == 0) continue;
         const int64_t blocks = std::min<int64_t>(sm_count(), acc);
-        rowquant_tma_kernel<<<(unsigned)blocks, kTmaThreads, smem, stream>>>(P);
+        rowquant_tma_kernel<kColScale><<<(unsigned)blocks, kTmaThreads, smem, stream>>>(P);
         if (launch_status() != GQ_OK) return GQ_ERR_CUDA;
     }
     return GQ_OK;
+}
+
+// Groups with AWQ column scales go to their own launch of the pipelined kernel.
+gq_status run_rows_tma(std::vector<RowDesc>& rows, cudaStream_t stream) {
+    std::vector<RowDesc> plain, scaled;
+    for (const RowDesc& D : rows) (D.colscale ? scaled : plain).push_back(D);
+    gq_status st = run_rows_tma_impl<false>(plain, stream);
+    if (st != GQ_OK) return st;
+    return run_rows_tma_impl<true>(scaled, stream);
 }
 
 gq_status run_passthrough(const std::vector<PassDesc>& pd, cudaStream_t stream) {
@@ -429,7 +440,8 @@ gq_status quantize_batch(const gq_tensor* t, int n, Op op, bool f16_mode, void* 
             D.items = T.rows;
         }
         D.flags = flags;
-        if (tma_eligible(T, flags) && !T.col_scale)   // column-scaled rows: the row kernels
+        // column scales read as float4 by the pipelined kernel (else the row kernels)
+        if (tma_eligible(T, flags) && (!T.col_scale || (flags & kVecCol)))
             rows_tma.push_back(D);
         else if (T.cols <= 2048)
             rows_w.push_back(D);
