@@ -999,20 +999,19 @@ __device__ __forceinline__ void issue_tile(const TmaParams& P, int it, int& di, 
     }
 }
 
-// AWQ column scaling of a staged tile, in place: nr rows of `cols` elements
-// (row_bytes apart, cols a multiple of 4), element (r, c) becomes
+// AWQ column scaling of one staged row, in place: element c becomes
 // RN_dtype(w * t[c]) -- one binary32 multiply, rounded to nearest even bf16
-// for a bf16 weight.  Thread `tt` of `nth` takes every nth-th quad.
-__device__ __forceinline__ void scale_columns(uint32_t stage, int nr, uint32_t row_bytes, int cols, int dtype,
-                                              const float* t, int tt, int nth) {
+// for a bf16 weight.  Thread `tl` of the row's `lpr` threads takes quads
+// tl, tl + lpr, ... (cols a multiple of 4).  The caller syncs the row's
+// threads before they read the row, after a proxy fence that orders these
+// generic stores before the next bulk copy into the stage.
+__device__ __forceinline__ void scale_row(uint32_t row, int cols, int dtype, const float* t, int tl, int lpr) {
     const int qpr = cols >> 2;
-    const int nq = nr * qpr;
     const float4* t4 = reinterpret_cast<const float4*>(t);
-    for (int i = tt; i < nq; i += nth) {
-        const int rr = i / qpr, j = i - rr * qpr;
+    for (int j = tl; j < qpr; j += lpr) {
         const float4 c = __ldg(t4 + j);
         if (dtype == kF32) {
-            const uint32_t a = stage + (uint32_t)rr * row_bytes + 16u * (uint32_t)j;
+            const uint32_t a = row + 16u * (uint32_t)j;
             float v0, v1, v2, v3;
             asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
                          : "=f"(v0), "=f"(v1), "=f"(v2), "=f"(v3)
@@ -1022,17 +1021,19 @@ __device__ __forceinline__ void scale_columns(uint32_t stage, int nr, uint32_t r
                          "f"(__fmul_rn(v1, c.y)), "f"(__fmul_rn(v2, c.z)), "f"(__fmul_rn(v3, c.w))
                          : "memory");
         } else {
-            const uint32_t a = stage + (uint32_t)rr * row_bytes + 8u * (uint32_t)j;
+            const uint32_t a = row + 8u * (uint32_t)j;
             uint32_t x, y;
             asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(x), "=r"(y) : "r"(a) : "memory");
-            const uint32_t h0 = float_to_bf16_bits(__fmul_rn(__uint_as_float(x << 16), c.x));
-            const uint32_t h1 = float_to_bf16_bits(__fmul_rn(__uint_as_float(x & 0xFFFF0000u), c.y));
-            const uint32_t h2 = float_to_bf16_bits(__fmul_rn(__uint_as_float(y << 16), c.z));
-            const uint32_t h3 = float_to_bf16_bits(__fmul_rn(__uint_as_float(y & 0xFFFF0000u), c.w));
-            asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(h0 | (h1 << 16)), "r"(h2 | (h3 << 16))
+            const __nv_bfloat162 lo = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(x << 16), c.x),
+                                                            __fmul_rn(__uint_as_float(x & 0xFFFF0000u), c.y));
+            const __nv_bfloat162 hi = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(y << 16), c.z),
+                                                            __fmul_rn(__uint_as_float(y & 0xFFFF0000u), c.w));
+            asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(*reinterpret_cast<const uint32_t*>(&lo)),
+                         "r"(*reinterpret_cast<const uint32_t*>(&hi))
                          : "memory");
         }
     }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // kColScale: the launch's descriptors all carry AWQ column scales (a
@@ -1119,15 +1120,6 @@ rowquant_tma_kernel(const __grid_constant__ TmaParams P) {
         const uint32_t row_bytes = (uint32_t)(D.cols * (D.dtype == kF32 ? 4 : 2));
         uint32_t stage;   // opaque to the compiler, ordered after the wait (see lds_quad)
         asm volatile("mov.b32 %0, %1;" : "=r"(stage) : "r"(smem_base + (uint32_t)s * SB) : "memory");
-        if constexpr (kColScale) {
-            // AWQ: the tile becomes the column-scaled weight RN_dtype(w * t[c])
-            // in place before the team reads it.  The proxy fence orders these
-            // generic stores before the next bulk copy into the stage.
-            scale_columns(stage, nr, row_bytes, (int)D.cols, D.dtype, D.colscale,
-                          (warp - team * wpt) * 32 + lane, team_threads);
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            named_sync(team == 0 ? 0 : 15, team_threads);
-        }
         Slot T;
         T.init(lpr, warp, lane);
         const int slots = team_threads >> T.lg;          // slots of this tile-team
@@ -1138,12 +1130,23 @@ rowquant_tma_kernel(const __grid_constant__ TmaParams P) {
                 const int i = rd * slots + lslot;
                 const bool rv = i < nr;
                 const uint32_t row = stage + (uint32_t)(rv ? i : 0) * row_bytes;
+                if constexpr (kColScale) {
+                    // AWQ: the row becomes RN_dtype(w * t[c]) in place before its
+                    // threads read it (the slots of a warp run in lockstep)
+                    if (rv) scale_row(row, (int)D.cols, D.dtype, D.colscale, T.tl, lpr);
+                    __syncwarp();
+                }
                 if (D.dtype == kF32) process_row_sub<kF32>(D, r0 + i, row, T, rv);
                 else process_row_sub<kBF16>(D, r0 + i, row, T, rv);
             }
         } else {
             for (int i = lslot; i < nr; i += slots, ++seq) {
                 const uint32_t row = stage + (uint32_t)i * row_bytes;
+                if constexpr (kColScale) {
+                    scale_row(row, (int)D.cols, D.dtype, D.colscale, T.tl, lpr);
+                    if (T.G > 1) T.team_sync();
+                    else __syncwarp();
+                }
                 uint32_t* bc = bcast + T.slot * kBcastWords;
                 uint32_t* hs = hist + T.slot * 256;
                 if (D.dtype == kF32) process_row_team<kF32>(D, r0 + i, row, T, lists, bc, hs, seq);
