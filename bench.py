@@ -684,6 +684,39 @@ def run_gemm(args):
                       "alg_gbs": round((wbytes + 2 * M * K + 4 * M * N) / us / 1e3, 1)}), flush=True)
 
 
+def run_awq(args):
+    """The AWQ column-scaled int6 export alone (``--awq ROWS,COLS``): a bf16
+    synthetic weight, column scales from synthetic activation statistics,
+    p = 0.9999; ``warmup`` then ``steps`` calls timed with CUDA events.  An
+    entry point for profiling that kernel; it prints one JSON line of its own."""
+    import torch
+    from int6_int8_weight_b200 import gq
+    rows, cols = (int(v) for v in args.awq.split(","))
+    device = torch.device("cuda")
+    Wb = synth.draw_bandwidth_matrix(rows, cols, 0, device=device).to(torch.bfloat16)
+    t = torch.from_numpy(synth.awq_col_scales(np.random.default_rng(3), cols)).to(device)
+    dq = torch.empty_like(Wb)
+    pk = torch.empty(rows, gq.gq_packed_row_bytes(cols, 6), dtype=torch.uint8, device=device)
+    h16 = torch.empty(rows, dtype=torch.float16, device=device)
+    d = gq.GQTensor(w=Wb.data_ptr(), dtype=1, qbits=6, gran=0, reserved=0, rows=rows, cols=cols, ld=cols,
+                    p=0.9999, dq=dq.data_ptr(), codes=0, packed=pk.data_ptr(), scale_f16=h16.data_ptr(),
+                    scale_f32=0, clip=0, col_scale=t.data_ptr())
+    arr = gq._arr([d])
+    for _ in range(args.warmup):
+        gq.LIB.gq_export_pack(arr, 1, None, 0, None, None)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        gq.LIB.gq_export_pack(arr, 1, None, 0, None, None)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / max(args.steps, 1)
+    alg = rows * cols * 4.75 + 2 * rows + 4 * cols
+    print(json.dumps({"awq": f"bf16 {rows}x{cols} int6 p=0.9999", "ms_per_call": round(ms, 4),
+                      "alg_gbs": round(alg / ms / 1e6, 1)}), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -699,9 +732,14 @@ def main(argv=None):
                          "underscores for spaces, e.g. f32_16384x16384_int6")
     ap.add_argument("--gemm", default=None,
                     help="profile the dequant-on-load GEMM alone on M,N,K,QBITS (one JSON line of its own)")
+    ap.add_argument("--awq", default=None,
+                    help="profile the AWQ column-scaled bf16 int6 export alone on ROWS,COLS (one JSON line of its own)")
     args = ap.parse_args(argv)
     if args.gemm:
         run_gemm(args)
+        return
+    if args.awq:
+        run_awq(args)
         return
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
