@@ -1008,6 +1008,8 @@ __device__ __forceinline__ void issue_tile(const TmaParams& P, int it, int& di, 
 __device__ __forceinline__ void scale_row(uint32_t row, int cols, int dtype, const float* t, int tl, int lpr) {
     const int qpr = cols >> 2;
     const float4* t4 = reinterpret_cast<const float4*>(t);
+    // unrolled: several scale loads (L1 hits, but long-latency) in flight
+#pragma unroll 4
     for (int j = tl; j < qpr; j += lpr) {
         const float4 c = __ldg(t4 + j);
         if (dtype == kF32) {
