@@ -169,3 +169,32 @@ def test_other_argument_errors(gq):
 def test_last_cuda_error_starts_clear(gq):
     assert gq.LIB.gq_last_cuda_error() == 0
     assert gq.LIB.gq_last_cuda_error_string().decode() == "no error"
+
+
+def test_gemm_argument_errors_before_launch(gq):
+    """gq_gemm_dequant refuses bad arguments on the host, before any CUDA call
+    (fake device addresses are never dereferenced)."""
+    L = gq.LIB
+    X, P, S, Y = 0x100000, 0x200000, 0x300000, 0x400000
+    ok = [X, 4, 64, 64, P, S, 6, 8, Y, 8, None, None]
+    bad_cases = [
+        (dict(i=6, v=7), 1),            # qbits
+        (dict(i=1, v=-1), 1),           # M < 0
+        (dict(i=3, v=32), 1),           # ldx < K
+        (dict(i=9, v=4), 1),            # ldy < N
+        (dict(i=2, v=48, j=3, w=48), 2),  # K not a multiple of 64
+        (dict(i=0, v=X + 2), 3),        # activations not 16-byte aligned
+        (dict(i=4, v=P + 8), 3),        # packed codes not 16-byte aligned
+        (dict(i=8, v=Y + 4), 3),        # Y not 16-byte aligned
+        (dict(i=9, v=10), 3),           # ldy % 4 != 0
+        (dict(i=0, v=0), 1),            # null activations
+    ]
+    for case, code in bad_cases:
+        args = list(ok)
+        args[case["i"]] = case["v"]
+        if "j" in case:
+            args[case["j"]] = case["w"]
+        assert L.gq_gemm_dequant(*args) == code, (case, code)
+    empty = list(ok)
+    empty[1] = 0                        # M = 0: nothing to do, nothing launched
+    assert L.gq_gemm_dequant(*empty) == 0
