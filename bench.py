@@ -47,6 +47,7 @@ import synth  # noqa: E402
 METRIC = "weight GB/s through fused fake-quant+export and % of B200 HBM peak"
 UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
+SPEC_HBM_GBS = 8000.0          # B200 HBM3e data-sheet figure, reported beside the measured peak
 FALLBACK_BF16_TFLOPS = 1590.0
 WORKLOAD = ("bandwidth stress: fp32 16384x16384, 65536x4096, 262144x512 and bf16 copies "
             "(Student-t nu=3, std 0.02); per matrix int6 per-row p=0.9999 clip-select+"
@@ -135,17 +136,73 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
-def traffic_per_launch(kernel_hash):
-    """ncu DRAM bytes of one step's fused launches, if taken on this source."""
-    path = os.path.join(ROOT, "profiles", "rowquant_traffic.json")
+TRAFFIC_PATH = os.path.join(ROOT, "profiles", "rowquant_traffic.json")
+
+
+def traffic_per_launch(kernel_hash, calls):
+    """Average ncu DRAM bytes (read + write) of one full-size launch of the
+    step, scaled from the per-row traffic of a smaller capture of the same
+    launches (traffic grows with the rows a launch processes), if it was taken
+    on the current kernel sources; else (None, None)."""
     try:
-        with open(path) as f:
+        with open(TRAFFIC_PATH) as f:
             d = json.load(f)
     except Exception:
         return None, None
     if d.get("kernel_source_hash") != kernel_hash:
         return None, None
-    return d.get("traffic_bytes_per_step"), d
+    per = d.get("per_call", {})
+    tot = 0.0
+    for _, _, _, name in calls:
+        if name not in per:
+            return None, None
+        rows = int(name.split()[1].split("x")[0])
+        tot += per[name]["dram_bytes_per_row"] * rows
+    return tot / len(calls), d
+
+
+def record_traffic(csv_path, shrink):
+    """Turn the ncu CSV of one shrunken step (dram__bytes_read.sum,
+    dram__bytes_write.sum, gpu__time_duration.sum of the 12 fused launches,
+    in call order) into profiles/rowquant_traffic.json."""
+    import csv
+    rows = [r for r in csv.reader(open(csv_path)) if len(r) > 10]
+    H = rows[0]
+    iid, mi, vi, ki = H.index("ID"), H.index("Metric Name"), H.index("Metric Value"), H.index("Kernel Name")
+    per_id, names = {}, {}
+    for r in rows[1:]:
+        if "rowquant" not in r[ki]:
+            continue
+        per_id.setdefault(int(r[iid]), {})[r[mi]] = float(r[vi].replace(",", ""))
+    ids = sorted(per_id)
+    calls = []
+    for dt in ("f32", "bf16"):
+        for (R, Cc) in synth.BANDWIDTH_SHAPES:
+            for q in (6, 8):
+                calls.append((f"{dt} {R}x{Cc} int{q}", R // shrink, Cc, 4 if dt == "f32" else 2, q))
+    assert len(ids) == len(calls), (len(ids), len(calls))
+    per_call = {}
+    for i, (name, r_small, cols, esz, q) in zip(ids, calls):
+        m = per_id[i]
+        dram = m["dram__bytes_read.sum"] + m["dram__bytes_write.sum"]
+        prb = 3 * ((cols + 3) // 4) if q == 6 else cols
+        alg = r_small * (cols * 2 * esz + prb + 2)
+        per_call[name] = {"rows_captured": r_small, "dram_read_bytes": int(m["dram__bytes_read.sum"]),
+                          "dram_write_bytes": int(m["dram__bytes_write.sum"]),
+                          "algorithmic_bytes": int(alg), "traffic_over_algorithmic": round(dram / alg, 4),
+                          "dram_bytes_per_row": dram / r_small, "ns": m.get("gpu__time_duration.sum")}
+    out = {"kernel": "gq::rowquant_tma_kernel<false> (no column scales)",
+           "kernel_source_hash": kernel_source_hash(), "shrink": shrink, "per_call": per_call,
+           "note": (f"ncu dram__bytes_read.sum + dram__bytes_write.sum (1 pass) of each of the 12 fused "
+                    f"launches of one step with every matrix's rows divided by {shrink}; bench.py scales "
+                    "each launch's bytes per row to the full row count"),
+           "command": ("ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum "
+                       f"--clock-control none -k regex:rowquant -s 36 -c 12 --csv --log-file "
+                       f"gpurun_out/step_traffic.csv python bench.py --shrink {shrink} --steps 1 "
+                       "--warmup 3 --skip-cpu --skip-rows --no-e2e")}
+    with open(TRAFFIC_PATH, "w") as f:
+        json.dump(out, f, indent=1)
+    return out
 
 
 # ---------------------------------------------------------------- clocks --
@@ -223,14 +280,18 @@ REJECT = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
 class Workload:
     """The six matrices, their preallocated outputs and one descriptor per call."""
 
-    def __init__(self, gq, device, seed, only=None):
+    def __init__(self, gq, device, seed, only=None, shrink=1):
         """``only``: restrict to the calls whose name contains this text
-        (e.g. "f32 16384x16384 int6"), for profiling a single launch."""
+        (e.g. "f32 16384x16384 int6"), for profiling a single launch.
+        ``shrink``: divide every matrix's row count by this factor (a smaller
+        case of the same launches for counter captures; never a bench line)."""
         self.gq = gq
         self.mats = []
+        self.shrink = shrink
         want = []
         for dt in ("f32", "bf16"):
             for i, (r, c) in enumerate(synth.BANDWIDTH_SHAPES):
+                r = r // shrink
                 names = [f"{dt} {r}x{c} int{q}" for q in (6, 8)]
                 if only is None or any(only in nm for nm in names):
                     want.append((dt, i, r, c))
@@ -248,7 +309,7 @@ class Workload:
             rows, cols = W.shape
             esz = W.element_size()
             for qbits, p in ((6, 0.9999), (8, 1.0)):
-                name = f"{'f32' if esz == 4 else 'bf16'} {rows}x{cols} int{qbits}"
+                name = f"{'f32' if esz == 4 else 'bf16'} {rows * shrink}x{cols} int{qbits}"
                 if only is not None and only not in name:
                     continue
                 dq = torch.empty_like(W)
@@ -299,12 +360,15 @@ def flush_l2(buf):
 
 def measure_rows(gq, device, peak):
     """Each remaining operation of the path, timed alone with CUDA events
-    (median of reps; L2 flushed between reps when the working set fits L2)."""
+    (5 warm-ups, median of 50 reps; L2 flushed between reps when the working
+    set fits L2).  The model-shaped batches (the single 512x1536 matrix, the
+    9-layer export, the 11-layer training step, the 12-layer mixed-bit export)
+    also carry the single-threaded CPU oracle's time on the same inputs."""
     out = {}
     flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=device)   # 256 MiB
 
-    def timed(fn, reps=20, flush_between=False):
-        for _ in range(3):
+    def timed(fn, reps=50, flush_between=False):
+        for _ in range(5):
             fn()
         ts = []
         for _ in range(reps):
@@ -406,8 +470,22 @@ def measure_rows(gq, device, peak):
         del q, X, Y, Wh
 
     # model-shaped batched workloads (L2-resident: flushed between reps)
-    def batch(specs_arrays, export=True, per_tensor_override=None, name="", note=""):
-        descs, keep = [], []
+    def oracle_time(items, export):
+        """Single-threaded CPU oracle on the same tensors: (seconds, bytes)."""
+        import oracle
+        t0 = time.perf_counter()
+        nb = 0
+        for w, qbits, p, per_tensor in items:
+            if qbits == 16:
+                oracle.passthrough_f16(w)
+            else:
+                r = oracle.quantize(w, qbits, p, per_tensor=per_tensor, export=export)
+                assert r.status == 0
+            nb += w.size * w.itemsize
+        return time.perf_counter() - t0, nb
+
+    def batch(specs_arrays, export=True, per_tensor_override=None, name="", note="", ste=False):
+        descs, keep, host_items = [], [], []
         alg = inb = 0
         for spec, w in specs_arrays:
             W = torch.from_numpy(w).to(device) if isinstance(w, np.ndarray) else w
@@ -418,6 +496,10 @@ def measure_rows(gq, device, peak):
             rows, cols = W.shape
             esz = W.element_size()
             keep.append(W)
+            w_host = w if isinstance(w, np.ndarray) else W.cpu().numpy()
+            if w_host.dtype == np.int16:
+                w_host = w_host.view(np.uint16)
+            w_host = w_host.reshape(rows, cols)
             if spec.qbits == 16:
                 out16 = torch.empty((rows, cols), dtype=torch.float16, device=device)
                 keep.append(out16)
@@ -426,6 +508,7 @@ def measure_rows(gq, device, peak):
                                          packed=out16.data_ptr(), scale_f16=0, scale_f32=0, clip=0))
                 alg += rows * cols * (esz + 2)
                 inb += rows * cols * esz
+                host_items.append((w_host, 16, 1.0, False))
                 continue
             per_tensor = spec.per_tensor if per_tensor_override is None else per_tensor_override
             prb = gq.gq_packed_row_bytes(cols, spec.qbits)
@@ -440,6 +523,7 @@ def measure_rows(gq, device, peak):
                                      scale_f16=h.data_ptr() if export else 0, scale_f32=0, clip=0))
             alg += rows * cols * 2 * esz + (rows * prb + 2 * rows if export else 0)
             inb += rows * cols * esz
+            host_items.append((w_host, spec.qbits, spec.p, per_tensor))
         arr = gq._arr(descs)
         nbytes = gq.gq_workspace_size(descs)
         ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
@@ -448,8 +532,59 @@ def measure_rows(gq, device, peak):
             fn = lambda: gq.LIB.gq_export_pack(arr, len(descs), ws.data_ptr(), ws.numel(), None, None)  # noqa: E731
         else:
             fn = lambda: gq.LIB.gq_fakequant_fwd(arr, len(descs), 0, ws.data_ptr(), ws.numel(), None, None)  # noqa: E731
+        launches = None
+        if ste:
+            # the STE backward of the same step: one flat gradient buffer for
+            # all weights (bf16 N(0, 1e-3^2)), copied to the weight gradient
+            numel = sum(int(np.prod(d.rows * d.cols)) for d in descs)
+            g_flat = (torch.randn(numel, device=device) * 1e-3).to(torch.bfloat16)
+            gw_flat = torch.empty_like(g_flat)
+            keep += [g_flat, gw_flat]
+            fwd = fn
+
+            def fn():
+                fwd()
+                gq.gq_ste_bwd(g_flat.data_ptr(), gw_flat.data_ptr(), 1, numel, 0)
+            alg += 4 * numel
         t = timed(fn, flush_between=True)
-        record(name, t, alg, inb, None, note)
+        record(name, t, alg, inb, launches, note)
+        cs, cb = oracle_time(host_items, export)
+        if ste:
+            import oracle
+            g_host = g_flat.cpu().view(torch.int16).numpy().view(np.uint16)
+            t0 = time.perf_counter()
+            oracle.ste_bwd(g_host)
+            cs += time.perf_counter() - t0
+        out[name]["cpu_oracle"] = {"gbs": round(cb / cs / 1e9, 4), "seconds": round(cs, 3), "cores": 1,
+                                   "kind": "oracle", "sample": "the whole batch, single-threaded C oracle"}
+
+    # the single 512x1536 fp32 matrix: int6 absmax export (w_hat, codes,
+    # packed, binary16 scales) + STE copy of a same-shape gradient
+    w0, g0 = synth.draw_single_matrix()
+    W0, G0 = torch.from_numpy(w0).to(device), torch.from_numpy(g0).to(device)
+    dq0, cd0 = torch.empty_like(W0), torch.empty(W0.shape, dtype=torch.int8, device=device)
+    pk0 = torch.empty(512, gq.gq_packed_row_bytes(1536, 6), dtype=torch.uint8, device=device)
+    h0, gw0 = torch.empty(512, dtype=torch.float16, device=device), torch.empty_like(G0)
+    arr0c = gq._arr([gq.GQTensor(w=W0.data_ptr(), dtype=0, qbits=6, gran=0, reserved=0, rows=512, cols=1536,
+                                 ld=1536, p=1.0, dq=dq0.data_ptr(), codes=cd0.data_ptr(), packed=pk0.data_ptr(),
+                                 scale_f16=h0.data_ptr(), scale_f32=0, clip=0)])
+
+    def c0():
+        gq.LIB.gq_export_pack(arr0c, 1, None, 0, None, None)
+        gq.gq_ste_bwd(G0.data_ptr(), gw0.data_ptr(), 0, 512 * 1536, 0)
+    n0 = 512 * 1536
+    record("single 512x1536 export int6 absmax + STE", timed(c0, flush_between=True),
+           n0 * (4 + 4 + 1 + 0.75) + 2 * 512 + 8 * n0, 4 * n0 + 4 * n0, 2,
+           note="cold L2; w_hat, codes, packed, fp16 scales + STE copy")
+    import oracle
+    t0 = time.perf_counter()
+    oracle.quantize(w0, 6, 1.0, export=True)
+    oracle.ste_bwd(g0)
+    cs0 = time.perf_counter() - t0
+    out["single 512x1536 export int6 absmax + STE"]["cpu_oracle"] = {
+        "gbs": round(8 * n0 / cs0 / 1e9, 4), "seconds": round(cs0, 3), "cores": 1, "kind": "oracle",
+        "sample": "the whole matrix and gradient, single-threaded C oracle"}
+    del W0, G0, dq0, cd0, pk0, h0, gw0
 
     ws9 = synth.draw_gpt9()
     batch([(s, ws9[s.name]) for s in synth.gpt9_specs()], name="gpt9 export batched (55 matrices + 27 fp16)",
@@ -463,7 +598,8 @@ def measure_rows(gq, device, peak):
           name="gpt12 int6 per-tensor p=.999 batched", note="cold L2; 3 select passes + quantize pass")
     wsu = synth.draw_unified11()
     batch([(s, wsu[s.name].view(np.int16)) for s in synth.unified11_train().specs], export=False,
-          name="unified11 bf16 train fake-quant batched", note="cold L2; w_hat only, fp32 scales")
+          name="unified11 bf16 train step: fake-quant batched + STE", ste=True,
+          note="cold L2; one iteration: w_hat (fp32 scales) of the 44 weights + STE copy of their gradients")
     torch.cuda.synchronize()
     return out
 
@@ -476,7 +612,7 @@ def run_ours(args, world, rank, local):
     peak, peak_kind = hbm_peak()
 
     only = args.only.replace("_", " ") if args.only else None
-    wl = Workload(gq, device, seed=4 + rank, only=only)
+    wl = Workload(gq, device, seed=4 + rank, only=only, shrink=args.shrink)
     handle = torch.cuda.current_stream(device).cuda_stream
     ncalls = len(wl.calls)
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * ncalls)] for _ in range(args.steps)]
@@ -503,14 +639,15 @@ def run_ours(args, world, rank, local):
             per_call[i] += dt
             launch_s += dt
     achieved = wl.alg_bytes * args.steps / launch_s / 1e9
-    traffic_step, tinfo = traffic_per_launch(kernel_source_hash())
+    traffic_launch, tinfo = traffic_per_launch(kernel_source_hash(), wl.calls)
     traffic = None
-    if traffic_step is not None and tinfo.get("launches_per_step") == ncalls and not args.only:
-        traffic = int(traffic_step / ncalls)
+    if traffic_launch is not None and not args.only and args.shrink == 1:
+        traffic = int(traffic_launch)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "peak_source": peak_kind,
+                "frac_of_spec": round(achieved / SPEC_HBM_GBS, 4), "spec_gbs": SPEC_HBM_GBS,
                 "traffic": traffic, "algorithmic_bytes_per_launch": int(wl.alg_bytes / ncalls),
-                "kernel": "rowquant_kernel (fused clip-select + quantize + dequant + pack), all "
+                "kernel": "rowquant_tma_kernel (fused clip-select + quantize + dequant + pack), all "
                           f"{ncalls} launches of a step",
                 "algorithmic_bytes_per_step": wl.alg_bytes,
                 "per_launch": {wl.calls[i][3]: {"ms": round(per_call[i] / args.steps * 1e3, 4),
@@ -542,6 +679,7 @@ def run_ours(args, world, rank, local):
                        "input_bytes_per_step": wl.in_bytes, "l2": "inputs larger than L2 (256 MiB-1 GiB each)",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
             "hbm_frac_step": round(wl.alg_bytes * args.steps / t_max / 1e9 / peak, 4),
+            "hbm_frac_step_of_spec": round(wl.alg_bytes * args.steps / t_max / 1e9 / SPEC_HBM_GBS, 4),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
             "gpu_launches": ncalls * args.steps, "rows": rows_extra,
         }
@@ -553,27 +691,70 @@ def run_ours(args, world, rank, local):
 
 def measure_e2e(gq, wl, device, world, handle, steps):
     """Same metric with the inputs copied in from pinned host memory and the
-    exported artifact (packed codes + binary16 scales) copied back, each step."""
+    exported artifact (packed codes + binary16 scales) copied back, each step.
+
+    Three streams overlap the work matrix by matrix: the host-to-device copy
+    of matrix i+1 and the device-to-host copy of matrix i-1's artifact run
+    while matrix i is quantized.  Events keep every buffer's reuse in order:
+    a matrix is not overwritten before the previous step's calls on it have
+    finished, and its outputs are not rewritten before they have been copied
+    back."""
     host_in = [W.cpu().pin_memory() for W in wl.mats]
     host_out = [(p.cpu().pin_memory(), h.cpu().pin_memory()) for (_, p, h) in wl.outs]
     h2d = sum(t.numel() * t.element_size() for t in host_in)
     d2h = sum(p.numel() + h.numel() * 2 for p, h in host_out)
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    s_cmp = torch.cuda.current_stream(device)
+    nm = len(wl.mats)
+    calls_of = [[] for _ in range(nm)]
+    for ci in range(len(wl.calls)):
+        calls_of[ci // 2].append(ci)          # two calls (int6, int8) per matrix, in order
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    done_cmp = [None] * nm                    # last compute on matrix i (its input is free)
+    done_out = [None] * nm                    # last copy-back of matrix i's outputs
 
     def one(_k):
-        for W, H in zip(wl.mats, host_in):
-            W.copy_(H, non_blocking=True)
-        wl.step(handle)
-        for (po, ho), (_, p, h) in zip(host_out, wl.outs):
-            po.copy_(p, non_blocking=True)
-            ho.copy_(h, non_blocking=True)
+        L = gq.LIB
+        for i in range(nm):
+            with torch.cuda.stream(s_in):
+                if done_cmp[i] is not None:
+                    s_in.wait_event(done_cmp[i])
+                wl.mats[i].copy_(host_in[i], non_blocking=True)
+                e_in = ev()
+                e_in.record(s_in)
+            s_cmp.wait_event(e_in)
+            if done_out[i] is not None:
+                s_cmp.wait_event(done_out[i])
+            for ci in calls_of[i]:
+                st = L.gq_export_pack(wl.calls[ci][0], 1, None, 0, None, handle)
+                if st != 0:
+                    raise RuntimeError(f"gq_export_pack failed: {st}")
+            done_cmp[i] = ev()
+            done_cmp[i].record(s_cmp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(done_cmp[i])
+                for ci in calls_of[i]:
+                    (po, ho), (_, p, h) = host_out[ci], wl.outs[ci]
+                    po.copy_(p, non_blocking=True)
+                    ho.copy_(h, non_blocking=True)
+                done_out[i] = ev()
+                done_out[i].record(s_out)
 
-    one(0)
-    elapsed = time_region(one, steps, world, device)
+    def joined(k):
+        one(k)
+        # the step ends when its last copy-back has landed
+        for e in done_out:
+            s_cmp.wait_event(e)
+
+    joined(0)
+    elapsed = time_region(joined, steps, world, device)
     v, _ = job_throughput(wl.in_bytes * steps, elapsed, world, device)
     del host_in, host_out
     return {"value": round(v / 1e9, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": steps,
-            "note": "pinned host weights -> device, libgq export calls, packed codes + fp16 scales -> host"}
+            "note": ("pinned host weights -> device, libgq export calls, packed codes + fp16 scales -> "
+                     "host; copies in, quantization and copies out overlap on three streams, matrix by "
+                     "matrix")}
 
 
 # ----------------------------------------------------------- CPU oracle --
@@ -732,9 +913,17 @@ def main(argv=None):
                          "underscores for spaces, e.g. f32_16384x16384_int6")
     ap.add_argument("--gemm", default=None,
                     help="profile the dequant-on-load GEMM alone on M,N,K,QBITS (one JSON line of its own)")
+    ap.add_argument("--shrink", type=int, default=1,
+                    help="divide every bandwidth matrix's rows by this factor (smaller case for ncu "
+                         "counter captures; its line is not a bench value)")
+    ap.add_argument("--record-traffic", default=None, metavar="CSV",
+                    help="write profiles/rowquant_traffic.json from the ncu CSV of a --shrink run")
     ap.add_argument("--awq", default=None,
                     help="profile the AWQ column-scaled bf16 int6 export alone on ROWS,COLS (one JSON line of its own)")
     args = ap.parse_args(argv)
+    if args.record_traffic:
+        print(json.dumps(record_traffic(args.record_traffic, args.shrink), indent=1))
+        return
     if args.gemm:
         run_gemm(args)
         return

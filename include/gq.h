@@ -266,8 +266,10 @@ GQ_API gq_status gq_export_pack(const gq_tensor* t, int n, void* d_ws,
  *  - At most GQ_NOALLOC_MAX_PER_TENSOR per-tensor descriptors per call; a
  *    larger batch returns GQ_ERR_WORKSPACE before anything is launched.
  *  - The first call on a device looks up the array's device address (with
- *    that device current) and caches it; make that first call before any
- *    stream capture.
+ *    that device current) and caches it until the process exits; make that
+ *    first call before any stream capture.  cudaDeviceReset unloads the
+ *    library's device code, which makes the cached address stale: do not
+ *    call this entry point on a device after resetting it.
  *  - All calls on a device share the one array and each call clears the part
  *    it uses; calls whose work overlaps on the GPU (different streams, or
  *    different host threads without ordering) race on it.
@@ -316,6 +318,72 @@ GQ_API gq_status gq_dequant(const uint8_t* d_packed, const uint16_t* d_scale_f16
 GQ_API gq_status gq_gemm_dequant(const void* d_x, int64_t M, int64_t K, int64_t ldx, const uint8_t* d_packed,
                                  const uint16_t* d_scale_f16, int qbits, int64_t N, float* d_y, int64_t ldy,
                                  int32_t* d_status, cudaStream_t stream);
+
+/*
+ * TEST HOOK, not for production use: exercises the timeout path of the bounded
+ * waits of the pipelined row kernel (the kernel behind gq_row_clip_select,
+ * gq_fakequant_fwd, gq_fakequant_average and gq_export_pack for rows that
+ * are 16-byte aligned with a pitch that is a multiple of 16 bytes).  The next
+ * launch of that kernel from the calling host thread (and only that one)
+ * gives its tile number `tile` (counted over the launch's descriptors, in
+ * order) a copy that announces 16 bytes more than it transfers, so that
+ * tile's barrier never completes although every issued copy does, and gives
+ * up every wait after wait_ns nanoseconds (1e6 .. 4e9).  The launch then sets
+ * GQ_STATUS_TIMEOUT in the status word of the descriptor that owns the tile
+ * it was on, ends, and leaves the library usable; outputs of that call are
+ * unspecified.  If no such launch follows, the hook stays armed.
+ * GQ_ERR_INVALID_ARG for tile < 0 or wait_ns outside that range.
+ * The pages have no counterpart: this is a test of the library's own
+ * failure handling.
+ */
+GQ_API gq_status gq_test_arm_wait_expiry(int64_t tile, uint64_t wait_ns);
+
+/*
+ * GPTQ-lite: int6 / int8 export of one weight W [rows, cols] (rows = output
+ * features, cols = inputs) in which each column's codes absorb the rounding
+ * error of the columns before it, weighted by the Hessian H of the layer's
+ * inputs.  Source: "Record: Unified Attention + FA3 + Legal TTT" (PR #1202),
+ * section Quantization: "GPTQ-lite", bits 6, scope weights.  The page gives no
+ * algorithm; this is the published GPTQ algorithm (Frantar et al., 2022,
+ * Algorithm 1) on the export's per-row grid:
+ *   - scales: exactly those of gq_export_pack on W (percentile clip of each
+ *     ORIGINAL row, s = binary16(c / qmax)); GPTQ changes only the codes;
+ *   - inputs whose diagonal H[j, j] is 0 are dead: H[j, j] is taken as 1 and
+ *     column j of W as 0; then lambda = percdamp * mean(diag H) is added to
+ *     the diagonal (the usual percdamp is 0.01);
+ *   - columns are quantized left to right; column j is rounded from
+ *     w~_j = w_j + sum_{i<j} (w_i - q_i s) V[i, j] / V[j, j], where V is the
+ *     upper-triangular factor with H = V V^T (V^-1 is the upper Cholesky factor
+ *     of H^-1 that the algorithm feeds its errors through), by the export's
+ *     quantizer: clip to +-c, divide by s, round half to even, clamp;
+ *   - all of it in binary64.
+ * Arguments:
+ *   t        one descriptor: GQ_PER_ROW, qbits 6 or 8, no col_scale, cols at
+ *            most 5800; packed and scale_f16 required; dq (q * s in w's
+ *            dtype), codes and clip optional; scale_f32 ignored
+ *   d_H      device binary64 [cols, cols], symmetric (e.g. from
+ *            gq_gptq_hessian), read only
+ *   percdamp damping fraction, >= 0
+ *   d_ws     device workspace of gq_gptq_workspace_size(rows, cols) bytes,
+ *            256-byte aligned (clip per row, dead flags, the Cholesky factor)
+ *   d_status nullable, one int32: cleared, then GQ_STATUS_NONFINITE for a
+ *            non-finite weight or a Hessian that is not positive definite
+ *            after damping, GQ_STATUS_RANGE for a binary16 scale overflow
+ * Asynchronous on `stream`; about 2 * cols / 64 + 5 kernel launches.
+ */
+GQ_API size_t gq_gptq_workspace_size(int64_t rows, int64_t cols);
+GQ_API gq_status gq_gptq_quantize(const gq_tensor* t, const double* d_H, double percdamp, void* d_ws,
+                                  size_t ws_bytes, int32_t* d_status, cudaStream_t stream);
+
+/*
+ * The Hessian of GPTQ-lite from calibration inputs: H = 2 X^T X (accumulate =
+ * 0) or H += 2 X^T X (accumulate = 1), binary64 [cols, cols], full symmetric.
+ * d_x is fp32 or bf16 (dtype) [n, ldx] row-major, one row per token, widened
+ * exactly; the products and sums are binary64.  The scale of H does not
+ * change the result of gq_gptq_quantize (its damping is relative).
+ */
+GQ_API gq_status gq_gptq_hessian(const void* d_x, int32_t dtype, int64_t n, int64_t cols, int64_t ldx,
+                                 double* d_H, int accumulate, cudaStream_t stream);
 
 /* Device workspace bytes a batch needs (0 when it has no per-tensor group). */
 GQ_API size_t gq_workspace_size(const gq_tensor* t, int n);

@@ -16,6 +16,7 @@
 
 #include "gq_aux_kernels.cuh"
 #include "gq_gemm.cuh"
+#include "gq_gptq.cuh"
 #include "gq_kernels.cuh"
 #include "gq_rowquant_tma.cuh"
 
@@ -193,6 +194,11 @@ gq_status run_rows(const std::vector<RowDesc>& rows, cudaStream_t stream) {
     return GQ_OK;
 }
 
+// Test hook of the bounded waits (gq_test_arm_wait_expiry): armed per host
+// thread, consumed by the next launch of the pipelined row kernel.
+thread_local int64_t g_test_poison_tile = -1;
+thread_local uint64_t g_test_wait_ns = 0;
+
 // Pipelined launch over the descriptors whose rows can be bulk-copied.
 constexpr int kTmaStageBytes = 68 * 1024;
 constexpr int kTmaMaxRowBytes = 96 * 1024;
@@ -286,6 +292,14 @@ gq_status run_rows_tma_impl(std::vector<RowDesc>& rows, cudaStream_t stream) {
         P.nstages = nstages;
         P.stage_bytes = sb;
         P.teams = teams;
+        P.wait_ns = kWaitLimitNs;
+        P.poison_tile = -1;
+        if (g_test_poison_tile >= 0) {
+            P.wait_ns = g_test_wait_ns;
+            P.poison_tile = g_test_poison_tile;
+            P.poison_bytes = 16;
+            g_test_poison_tile = -1;
+        }
         int64_t acc = 0;
         for (int i = 0; i < nd; ++i) {
             P.start[i] = acc;
@@ -521,9 +535,152 @@ gq_status noalloc_scratch(void** out) {
     return GQ_OK;
 }
 
+// ------------------------------------------------------------- GPTQ-lite --
+
+constexpr int64_t kGptqMaxCols = 5800;     // residual rows of a block stay in shared memory
+
+size_t round256(size_t v) { return (v + 255) / 256 * 256; }
+
+struct GptqWs {
+    float* clip;
+    uint8_t* dead;
+    GpState* st;
+    double* L;
+    size_t bytes;
+};
+
+GptqWs gptq_layout(void* base, int64_t rows, int64_t cols) {
+    GptqWs w{};
+    size_t off = 0;
+    auto take = [&](size_t b) {
+        size_t o = off;
+        off += round256(b);
+        return o;
+    };
+    const size_t o_clip = take((size_t)rows * 4), o_dead = take((size_t)cols), o_st = take(sizeof(GpState)),
+                 o_L = take((size_t)cols * (size_t)cols * 8);
+    unsigned char* b = static_cast<unsigned char*>(base);
+    if (b) {
+        w.clip = reinterpret_cast<float*>(b + o_clip);
+        w.dead = b + o_dead;
+        w.st = reinterpret_cast<GpState*>(b + o_st);
+        w.L = reinterpret_cast<double*>(b + o_L);
+    }
+    w.bytes = off;
+    return w;
+}
+
+std::atomic<int> g_gptq_smem_set[kMaxDevices];
+
 }  // namespace
 
 extern "C" {
+
+size_t gq_gptq_workspace_size(int64_t rows, int64_t cols) {
+    if (rows < 0 || cols < 0) return 0;
+    return gptq_layout(nullptr, rows, cols).bytes;
+}
+
+gq_status gq_gptq_hessian(const void* d_x, int32_t dtype, int64_t n, int64_t cols, int64_t ldx, double* d_H,
+                          int accumulate, cudaStream_t stream) {
+    if (dtype != GQ_F32 && dtype != GQ_BF16) return GQ_ERR_INVALID_ARG;
+    if (n < 0 || cols < 0 || ldx < cols || (accumulate != 0 && accumulate != 1)) return GQ_ERR_INVALID_ARG;
+    if (cols == 0) return GQ_OK;
+    if (!d_H || (n > 0 && !d_x)) return GQ_ERR_INVALID_ARG;
+    if (cols > 65535 * (int64_t)kGpHTile || (n > 0 && n > INT64_MAX / 4 / ldx)) return GQ_ERR_UNSUPPORTED;
+    if (!aligned(d_H, 8) || (n > 0 && !aligned(d_x, dtype == GQ_F32 ? 4 : 2))) return GQ_ERR_MISALIGNED;
+    const unsigned tiles = (unsigned)((cols + kGpHTile - 1) / kGpHTile);
+    gptq_hessian_kernel<<<dim3(tiles, tiles), kGpThreads, 0, stream>>>(d_x, dtype, n, cols, ldx, d_H, accumulate);
+    return launch_status();
+}
+
+gq_status gq_gptq_quantize(const gq_tensor* t, const double* d_H, double percdamp, void* d_ws, size_t ws_bytes,
+                           int32_t* d_status, cudaStream_t stream) {
+    if (!t) return GQ_ERR_INVALID_ARG;
+    const gq_tensor& T = *t;
+    gq_status st = check_tensor(T, Op::Export, true);
+    if (st != GQ_OK) return st;
+    if (T.qbits == 16 || T.gran != GQ_PER_ROW || T.col_scale) return GQ_ERR_UNSUPPORTED;
+    if (!(percdamp >= 0.0 && percdamp < 1e6)) return GQ_ERR_INVALID_ARG;
+    if (d_status && !aligned(d_status, 4)) return GQ_ERR_MISALIGNED;
+    if (T.rows == 0 || T.cols == 0) {
+        if (d_status) return cuda_status(cudaMemsetAsync(d_status, 0, sizeof(int32_t), stream));
+        return GQ_OK;
+    }
+    if (!d_H) return GQ_ERR_INVALID_ARG;
+    if (!aligned(d_H, 8)) return GQ_ERR_MISALIGNED;
+    if (T.cols > kGptqMaxCols) return GQ_ERR_UNSUPPORTED;
+    const GptqWs W = gptq_layout(d_ws, T.rows, T.cols);
+    if (!d_ws || ws_bytes < W.bytes) return GQ_ERR_WORKSPACE;
+    if (!aligned(d_ws, 256)) return GQ_ERR_MISALIGNED;
+    const int64_t n = T.cols;
+
+    // 1. clip of every original row (the export's select), into the workspace
+    gq_tensor sel = T;
+    sel.dq = nullptr;
+    sel.codes = nullptr;
+    sel.packed = nullptr;
+    sel.scale_f16 = nullptr;
+    sel.scale_f32 = nullptr;
+    sel.clip = W.clip;
+    st = quantize_batch(&sel, 1, Op::Select, false, nullptr, 0, d_status, stream);
+    if (st != GQ_OK) return st;
+    if (T.clip && cuda_status(cudaMemcpyAsync(T.clip, W.clip, (size_t)T.rows * 4, cudaMemcpyDeviceToDevice,
+                                              stream)) != GQ_OK)
+        return GQ_ERR_CUDA;
+    // 2. dead inputs, damping, reversal
+    gptq_diag_kernel<<<1, kGpThreads, 0, stream>>>(d_H, n, percdamp, W.dead, W.st);
+    const int64_t rev_blocks = std::min<int64_t>((int64_t)sm_count() * 8, (n * n + kGpThreads - 1) / kGpThreads);
+    gptq_reverse_kernel<<<(unsigned)rev_blocks, kGpThreads, 0, stream>>>(d_H, n, W.dead, W.st, W.L);
+    if (launch_status() != GQ_OK) return GQ_ERR_CUDA;
+    // 3. Cholesky of the reversed, damped Hessian
+    for (int64_t k0 = 0; k0 < n; k0 += kGpBlock) {
+        const int64_t nb = std::min<int64_t>(kGpBlock, n - k0);
+        const int64_t below = n - k0 - nb;
+        const unsigned pblocks = (unsigned)std::max<int64_t>(1, (below + 63) / 64);
+        gptq_chol_panel<<<pblocks, kGpThreads, 0, stream>>>(W.L, n, k0, W.st);
+        if (below > 0) {
+            const unsigned ut = (unsigned)((below + 63) / 64);
+            gptq_chol_update<<<dim3(ut, ut), kGpThreads, 0, stream>>>(W.L, n, k0);
+        }
+        if (launch_status() != GQ_OK) return GQ_ERR_CUDA;
+    }
+    // 4. the recurrence over the rows
+    GptqParams P;
+    std::memset(&P, 0, sizeof(P));
+    P.ndesc = 1;
+    GptqRowDesc& R = P.d[0];
+    R.w = T.w;
+    R.L = W.L;
+    R.dead = W.dead;
+    R.st = W.st;
+    R.clip = W.clip;
+    R.scale_f16 = T.scale_f16;
+    R.codes = T.codes;
+    R.packed = T.packed;
+    R.dq = T.dq;
+    R.status = d_status;
+    R.rows = T.rows;
+    R.n = n;
+    R.ld = T.ld;
+    R.prb = packed_row_bytes(n, T.qbits);
+    R.start = 0;
+    R.dtype = T.dtype;
+    R.qbits = T.qbits;
+    P.blocks = (T.rows + kGpRows - 1) / kGpRows;
+    if (P.blocks > INT32_MAX) return GQ_ERR_UNSUPPORTED;
+    const size_t smem = gptq_rows_smem(n);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GQ_ERR_CUDA;
+    if (dev >= 0 && dev < kMaxDevices && g_gptq_smem_set[dev].load() < (int)smem) {
+        if (cuda_status(cudaFuncSetAttribute(gptq_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem)) != GQ_OK)
+            return GQ_ERR_CUDA;
+        g_gptq_smem_set[dev].store((int)smem);
+    }
+    gptq_rows_kernel<<<(unsigned)P.blocks, kGpThreads, smem, stream>>>(P);
+    return launch_status();
+}
 
 gq_status gq_row_clip_select(const gq_tensor* t, int n, void* d_ws, size_t ws_bytes,
                              int32_t* d_status, cudaStream_t stream) {
@@ -559,6 +716,13 @@ gq_status gq_export_pack_noalloc(const gq_tensor* t, int n, int32_t* d_status,
         if (st != GQ_OK) return st;
     }
     return quantize_batch(t, n, Op::Export, true, ws, kNoAllocBytes, d_status, stream);
+}
+
+gq_status gq_test_arm_wait_expiry(int64_t tile, uint64_t wait_ns) {
+    if (tile < 0 || wait_ns < 1000000ull || wait_ns > kWaitLimitNs) return GQ_ERR_INVALID_ARG;
+    g_test_poison_tile = tile;
+    g_test_wait_ns = wait_ns;
+    return GQ_OK;
 }
 
 gq_status gq_ste_bwd(const void* d_g_out, void* d_g_w, gq_dtype dtype, int64_t numel,

@@ -1,30 +1,44 @@
 // gq_rowquant_tma.cuh -- the fused per-row kernel, pipelined through shared
 // memory with bulk asynchronous copies (sm_100a).
 //
-// One persistent block per SM: warp 16 is the producer, warps 0..15 consume.
+// One persistent 512-thread block (16 warps) per SM and no producer warp.
 // The weights are cut into tiles of whole rows (one descriptor per tile) that
-// fill a stage of a ring of shared-memory stages.  The producer's elected lane
-// issues cp.async.bulk copies global -> shared for the next tiles while the
-// consumers work on the current one; completion is tracked by one mbarrier per
-// stage ("full", transaction bytes) and stages are handed back through a
-// second mbarrier ("empty", one arrival per consumer warp).  Each input byte
-// is read from HBM exactly once, with up to (stages - 1) tiles in flight.
+// fill the stages of a ring in shared memory.  Thread 0 issues the first fill
+// of every stage; after that the stage's last reader refills it:
+//   - fill k of stage s completes phase k / 2 of full[2 s + k % 2] (two
+//     "full" mbarriers per stage used on alternate fills, transaction bytes),
+//     so a one-bit parity wait is never ambiguous for a reader that lags one
+//     fill behind;
+//   - done[s] counts the warps that have finished with stage s (an
+//     acquire-release shared-memory atomic per warp); every fill is read by
+//     one tile-team of wpt warps, so the warp whose increment makes the count
+//     a multiple of wpt is the fill's last reader, and its lane 0 issues the
+//     next cp.async.bulk copy into the stage.
+// With three stages the 16 warps form two tile-teams of 8 that take
+// alternate tiles.  Each input byte is read from HBM exactly once.
 //
-// A row is owned by a slot of `lpr` consumer threads (lanes per row, a power
-// of two from 8 to 512, chosen per descriptor):
-//   lpr <= 32 : 32 / lpr rows share a warp, so every per-row step (the
+// A row is owned by a slot of `lpr` threads of a tile-team (lanes per row, a
+// power of two from 8 to 512, chosen per descriptor):
+//   lpr <= 16 : 32 / lpr rows share a warp, so every per-row step (the
 //               selection butterfly, the scale, the output pointers) is one
 //               warp instruction for several rows;
-//   lpr >= 64 : G = lpr / 32 warps own a row; the first warp merges the
-//               per-warp selections and broadcasts the row's clip through
-//               shared memory (two team barriers per row).
+//   lpr >= 32 : G = lpr / 32 warps own a row; each publishes its top-m list
+//               in shared memory, the row's warps meet at a named barrier and
+//               every warp merges the lists.
 // The row is read from shared memory twice (selection, then quantize), and
 // every output (w_hat, int8 codes, packed int6 / int8 bytes, scales) is
 // written from registers with coalesced vector stores.
 //
-// Every wait is bounded (a few seconds of %globaltimer): on expiry the thread
-// records GQ_STATUS_TIMEOUT in the tile's status word and leaves its loop; the
-// producer first waits, again bounded, for the copies it issued.  No wait is
+// Every wait on a full barrier is bounded (4 s of %globaltimer unless the
+// launch sets a shorter limit).  A warp whose wait gives up enters abort mode:
+// it records GQ_STATUS_TIMEOUT in the status word of every tile it still
+// touches, no longer waits, issues no refill, but still walks its
+// tile-team's tiles with the same control flow, so that every named barrier
+// the team meets is met by all of its warps (a warp that left would leave
+// the others waiting at such a barrier forever).  Its tile-mates then give up
+// at the first fill that the aborted warp would have started.  Before the
+// block exits, thread 0 waits (bounded) for the last fill issued into every
+// stage, so that no copy is still landing in shared memory.  No wait is
 // expected to expire; the bound keeps a defect from hanging the GPU.
 #pragma once
 
@@ -50,6 +64,13 @@ struct TmaParams {
     int32_t stage_bytes;
     int32_t teams;       // tile-teams: the consumer warps split into `teams` groups
                          // that take alternate tiles (1 or 2)
+    uint64_t wait_ns;    // limit of every bounded wait (kWaitLimitNs normally)
+    // Test hook for the timeout path: the copy of global tile poison_tile
+    // (-1: none) announces poison_bytes more bytes than it transfers, so its
+    // full barrier never completes although every issued copy does.
+    int64_t poison_tile;
+    uint32_t poison_bytes;
+    uint32_t pad_;
     int64_t start[kMaxDesc + 1];   // prefix sums of tiles
     RowDesc d[kMaxDesc];
 };
@@ -57,7 +78,7 @@ struct TmaParams {
 // Shared memory after the stages: mbarriers and stage counters, per-warp
 // selection lists, per-slot broadcast records and per-slot radix histograms.
 constexpr int kBcastWords = 8;
-constexpr int kTmaExtraBytes = 3 * kTmaMaxStages * 8 + 2 * kTmaConsumerWarps * kTopMax * 4 +
+constexpr int kTmaExtraBytes = 4 * kTmaMaxStages * 8 + 2 * kTmaConsumerWarps * kTopMax * 4 +
                                kTmaConsumerWarps * kBcastWords * 4 + kTmaConsumerWarps * 256 * 4;
 
 // ------------------------------------------------------------- PTX glue --
@@ -105,14 +126,16 @@ __device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t addr, uint32_t v) 
 }
 
 // Bounded wait for the completion of the phase with the given parity.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned long long limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 255u) == 0u && global_ns() - t0 > kWaitLimitNs) return false;
+        if ((i & 255u) == 0u && global_ns() - t0 > limit_ns) return false;
     }
 }
+
+
 
 // Bulk copy global -> this CTA's shared memory, completing `bytes` on `bar`.
 // Both addresses 16-byte aligned, bytes a multiple of 16.
@@ -991,7 +1014,7 @@ __device__ __forceinline__ void issue_tile(const TmaParams& P, int it, int& di, 
     const uint32_t row_bytes = (uint32_t)(D.cols * esz);
     const uint32_t dst = smem_base + (uint32_t)(it % S) * SB;
     const char* src = reinterpret_cast<const char*>(D.w) + r0 * D.ld * esz;
-    mbar_arrive_expect_tx(bar, (uint32_t)nr * row_bytes);
+    mbar_arrive_expect_tx(bar, (uint32_t)nr * row_bytes + (t == P.poison_tile ? P.poison_bytes : 0u));
     if (D.ld == D.cols) {
         bulk_g2s(dst, src, (uint32_t)nr * row_bytes, bar);
     } else {
@@ -1058,9 +1081,13 @@ rowquant_tma_kernel(const __grid_constant__ TmaParams P) {
     // increment makes the count a multiple of wpt is the last reader of the
     // fill and starts the next one.
     uint32_t* done = reinterpret_cast<uint32_t*>(full + 2 * kTmaMaxStages);
+    // last_fill[s]: the latest fill issued into stage s (-1: none), and the
+    // count of warps that have left the tile loop, for the drain before exit
+    int32_t* last_fill = reinterpret_cast<int32_t*>(done + kTmaMaxStages);
+    uint32_t* exited = reinterpret_cast<uint32_t*>(last_fill + kTmaMaxStages);
     auto full_bar = [&](int stage, int fill) { return smem_u32(&full[2 * stage + (fill & 1)]); };
     auto full_parity = [](int fill) { return (uint32_t)((fill >> 1) & 1); };
-    float* lists = reinterpret_cast<float*>(full + 3 * kTmaMaxStages);                     // [2][warp][kTopMax]
+    float* lists = reinterpret_cast<float*>(full + 4 * kTmaMaxStages);                     // [2][warp][kTopMax]
     uint32_t* bcast = reinterpret_cast<uint32_t*>(lists + 2 * kTmaConsumerWarps * kTopMax);  // [slot][8]
     uint32_t* hist = bcast + kTmaConsumerWarps * kBcastWords;                          // [slot][256]
 
@@ -1073,7 +1100,9 @@ rowquant_tma_kernel(const __grid_constant__ TmaParams P) {
             mbar_init(smem_u32(&full[2 * s]), 1);
             mbar_init(smem_u32(&full[2 * s + 1]), 1);
             done[s] = 0u;
+            last_fill[s] = blockIdx.x + (int64_t)s * gridDim.x < ntiles ? 0 : -1;
         }
+        *exited = 0u;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         // first fill of every stage
@@ -1093,6 +1122,7 @@ rowquant_tma_kernel(const __grid_constant__ TmaParams P) {
     int di = 0;           // tiles come in increasing order: their descriptors too
     int prev_lpr = 0;
     int seq = 0;          // rows this warp's slot has processed since the last shape change
+    bool aborted = false; // a wait of this warp gave up (warp-uniform)
     for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
         if (it % teams != team) continue;
         const int s = it % S;
@@ -1109,14 +1139,10 @@ rowquant_tma_kernel(const __grid_constant__ TmaParams P) {
             prev_lpr = lpr;
             seq = 0;
         }
-        if (!mbar_wait(full_bar(s, k), full_parity(k))) {
-            if (lane == 0) {
-                if (D.status) atomicOr(reinterpret_cast<unsigned int*>(D.status), kStatusTimeout);
-                // wait (bounded) for the copies that may still be in flight
-                for (int j = it; j < it + S; ++j) (void)mbar_wait(full_bar(j % S, j / S), full_parity(j / S));
-            }
-            break;
-        }
+        if (!aborted) aborted = !__all_sync(0xFFFFFFFFu, mbar_wait(full_bar(s, k), full_parity(k), P.wait_ns));
+        // abort mode: the tile is walked with the team (its barriers are met)
+        // but its stage may hold anything; its outputs are marked unspecified
+        if (aborted && lane == 0 && D.status) atomicOr(reinterpret_cast<unsigned int*>(D.status), kStatusTimeout);
         const int64_t r0 = (t - P.start[di]) * D.tile_rows;
         const int nr = (int)min((int64_t)D.tile_rows, D.rows - r0);
         const uint32_t row_bytes = (uint32_t)(D.cols * (D.dtype == kF32 ? 4 : 2));
@@ -1160,10 +1186,25 @@ rowquant_tma_kernel(const __grid_constant__ TmaParams P) {
         __syncwarp();
         if (lane == 0) {
             const uint32_t before = atom_add_acq_rel(smem_u32(&done[s]), 1u);
-            if ((before + 1u) % (uint32_t)wpt == 0u && t + (int64_t)S * gridDim.x < ntiles)
+            if ((before + 1u) % (uint32_t)wpt == 0u && t + (int64_t)S * gridDim.x < ntiles && !aborted) {
                 issue_tile(P, it + S, di_issue, smem_base, SB, S, full_bar(s, k + 1));
+                atomicMax(&last_fill[s], k + 1);
+            }
         }
     }
+    // No copy may still be landing when the block exits.  Only the latest
+    // fill of a stage can be incomplete: a later fill is issued only by a warp
+    // whose own wait saw the earlier one complete.  The last warp to leave
+    // the loop (no fill is issued after that) waits, bounded, for the latest
+    // fill of every stage; instant unless a wait gave up.  (No CTA-wide
+    // barrier here: a tile-team that is done must not meet the other team's
+    // shape-change barrier, which uses barrier 0 with a different count.)
+    __syncwarp();
+    if (lane == 0 && atom_add_acq_rel(smem_u32(exited), 1u) == (uint32_t)kTmaConsumerWarps - 1u)
+        for (int st = 0; st < S; ++st) {
+            const int f = atomicAdd(&last_fill[st], 0);
+            if (f >= 0) (void)mbar_wait(full_bar(st, f), full_parity(f), P.wait_ns);
+        }
 }
 
 }  // namespace gq

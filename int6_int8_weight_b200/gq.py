@@ -40,7 +40,8 @@ STATUS_NAMES = {0: "GQ_OK", 1: "GQ_ERR_INVALID_ARG", 2: "GQ_ERR_UNSUPPORTED",
 
 EXPORTED = ("gq_row_clip_select", "gq_fakequant_fwd", "gq_fakequant_average", "gq_ste_bwd", "gq_export_pack",
             "gq_export_pack_noalloc", "gq_dequant", "gq_gemm_dequant", "gq_workspace_size", "gq_packed_row_bytes", "gq_k_from_p",
-            "gq_plan_kind", "gq_status_string", "gq_last_cuda_error", "gq_last_cuda_error_string")
+            "gq_plan_kind", "gq_status_string", "gq_last_cuda_error", "gq_last_cuda_error_string",
+            "gq_test_arm_wait_expiry", "gq_gptq_quantize", "gq_gptq_hessian", "gq_gptq_workspace_size")
 
 
 class GQError(RuntimeError):
@@ -85,6 +86,14 @@ def _load() -> C.CDLL:
               "gq_export_pack_noalloc",
               "gq_ste_bwd", "gq_dequant", "gq_gemm_dequant"):
         getattr(L, f).restype = i32
+    L.gq_gptq_quantize.argtypes = [T, vp, f64, vp, sz, vp, vp]
+    L.gq_gptq_quantize.restype = i32
+    L.gq_gptq_hessian.argtypes = [vp, i32, i64, i64, i64, vp, i32, vp]
+    L.gq_gptq_hessian.restype = i32
+    L.gq_gptq_workspace_size.argtypes = [i64, i64]
+    L.gq_gptq_workspace_size.restype = sz
+    L.gq_test_arm_wait_expiry.argtypes = [i64, C.c_uint64]
+    L.gq_test_arm_wait_expiry.restype = i32
     L.gq_workspace_size.argtypes = [T, i32]
     L.gq_workspace_size.restype = sz
     L.gq_packed_row_bytes.argtypes = [i64, i32]
@@ -402,6 +411,44 @@ def gemm_dequant(x: torch.Tensor, packed: torch.Tensor, scale_f16: torch.Tensor,
     gq_gemm_dequant(x.data_ptr(), M, K, x.stride(0), packed.data_ptr(), scale_f16.data_ptr(), qbits, N,
                     y.data_ptr(), y.stride(0), 0, stream)
     return y
+
+
+def gptq_hessian(x: torch.Tensor, H: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """H = 2 X^T X (new fp64 tensor) or H += 2 X^T X (in place) for calibration
+    inputs ``x`` fp32 / bf16 [n, cols] with contiguous rows (GPTQ-lite)."""
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a 2-D [n, cols] tensor with contiguous rows")
+    n, cols = x.shape
+    accumulate = H is not None
+    if H is None:
+        H = torch.empty((cols, cols), dtype=torch.float64, device=x.device)
+    elif H.dtype != torch.float64 or H.shape != (cols, cols) or not H.is_contiguous():
+        raise ValueError("H must be a contiguous fp64 [cols, cols] tensor")
+    _check(LIB.gq_gptq_hessian(x.data_ptr(), _dtype_code(x), n, cols, x.stride(0), H.data_ptr(),
+                               int(accumulate), _stream(stream)), "gq_gptq_hessian")
+    return H
+
+
+def gptq_quantize(req: Request, H: torch.Tensor, percdamp: float = 0.01, stream=None,
+                  check_status: bool = True) -> Quantized:
+    """GPTQ-lite export of ``req.w`` (per row, qbits 6 / 8) against the fp64
+    Hessian ``H`` of its inputs; packed codes and binary16 scales are always
+    produced, the other outputs as requested."""
+    if req.per_tensor or req.qbits not in (6, 8) or req.col_scale is not None:
+        raise ValueError("GPTQ-lite takes per-row int6 / int8 requests without column scales")
+    r = Request(**{**req.__dict__, "want_packed": True, "want_scale_f16": True, "want_scale_f32": False})
+    (d,), (o,) = _prepare([r], True)
+    if H.dtype != torch.float64 or not H.is_contiguous() or H.shape != (d.cols, d.cols):
+        raise ValueError("H must be a contiguous fp64 [cols, cols] tensor")
+    dev = req.w.device
+    nbytes = LIB.gq_gptq_workspace_size(d.rows, d.cols)
+    ws = _SCRATCH.workspace(dev, nbytes)
+    st = _SCRATCH.status(dev, 1)
+    _check(LIB.gq_gptq_quantize(C.byref(d), H.data_ptr(), float(percdamp), ws.data_ptr(), ws.numel(),
+                                st.data_ptr(), _stream(stream)), "gq_gptq_quantize")
+    if check_status:
+        o.status = int(st[0].item())
+    return o
 
 
 def ste_bwd(g_out: torch.Tensor, g_w: torch.Tensor | None = None, stream=None) -> torch.Tensor:

@@ -256,3 +256,29 @@ def awq_col_scales(rng, cols):
     a = np.abs(rng.standard_normal(cols)) * np.exp(1.5 * rng.standard_normal(cols)) + 1e-3
     r = np.sqrt(a)
     return (r / math.sqrt(r.max() * r.min())).astype(np.float32)
+
+
+def gptq_calibration(rng, n, cols, rho=0.8, dead=()):
+    """Synthetic layer inputs for GPTQ-lite calibration: fp32 [n, cols], one
+    row per token.  Neighbouring features are correlated (AR(1) with
+    coefficient ``rho`` across the feature index) and every feature has its
+    own log-normal magnitude (a few large-activation channels), as the inputs
+    of a transformer layer have.  Columns listed in ``dead`` are zero (inputs
+    that are never active)."""
+    z = rng.standard_normal((n, cols))
+    x = np.empty_like(z)
+    x[:, 0] = z[:, 0]
+    k = math.sqrt(1.0 - rho * rho)
+    for j in range(1, cols):
+        x[:, j] = rho * x[:, j - 1] + k * z[:, j]
+    x *= np.exp(0.5 * rng.standard_normal(cols))[None, :]
+    for j in dead:
+        x[:, j] = 0.0
+    return x.astype(np.float32)
+
+
+def unified11_gptq_inputs():
+    """Per layer of the 11-layer d528 model, the input dimension of each of its
+    four weights (unified projection, out-projection, MLP up, MLP down), in the
+    order of unified11_train().specs."""
+    return [s.shape[1] for s in unified11_train().specs]

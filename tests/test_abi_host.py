@@ -198,3 +198,10 @@ def test_gemm_argument_errors_before_launch(gq):
     empty = list(ok)
     empty[1] = 0                        # M = 0: nothing to do, nothing launched
     assert L.gq_gemm_dequant(*empty) == 0
+
+
+def test_wait_expiry_hook_rejects_bad_arguments(gq):
+    # host-only: a rejected request arms nothing and launches nothing
+    assert gq.LIB.gq_test_arm_wait_expiry(-1, 5_000_000) == 1
+    assert gq.LIB.gq_test_arm_wait_expiry(0, 999_999) == 1
+    assert gq.LIB.gq_test_arm_wait_expiry(0, 4_000_000_001) == 1

@@ -7,7 +7,8 @@ For them gq_export_pack_noalloc takes its per-tensor scratch from a fixed
 array inside libgq.  This test calls it through the C ABI and checks that its
 outputs equal those of gq_export_pack (bit for bit, the tolerance of every
 parity test here) on two calls in a row with different inputs, so that what
-the first call leaves in the shared array cannot leak into the second.
+the first call leaves in the shared array cannot leak into the second; the
+outputs are also checked against the CPU oracle.
 
 The file is named so that pytest collects it last; it must also pass alone in
 a fresh process (the first call on the device sets the array up).
@@ -18,6 +19,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import synth
 
 pytestmark = pytest.mark.gpu
@@ -85,6 +87,21 @@ def test_noalloc_matches_export_on_two_calls(gq):
         for i, (g, w) in enumerate(zip(got, want)):
             for name, x, y in zip(("dq", "codes", "packed", "scale_f16", "clip"), g, w):
                 assert _same(x, y), (call, i, name)
+        for i, (W, d, g) in enumerate(zip(mats, got_descs, got)):
+            w_host = W.cpu()
+            w_np = (w_host.view(torch.int16).numpy().view(np.uint16) if W.dtype == torch.bfloat16
+                    else w_host.numpy())
+            ref = oracle.quantize(w_np, d.qbits, d.p, per_tensor=d.gran == 1, export=True)
+            assert ref.status == 0
+            dq_np = g[0].cpu()
+            dq_np = (dq_np.view(torch.int16).numpy().view(np.uint16) if W.dtype == torch.bfloat16
+                     else dq_np.numpy().view(np.uint32))
+            want_dq = ref.dq.view(np.uint32) if ref.dq.dtype == np.float32 else ref.dq
+            assert np.array_equal(dq_np, want_dq), (call, i, "dq vs oracle")
+            assert np.array_equal(g[1].cpu().numpy(), ref.codes), (call, i, "codes vs oracle")
+            assert np.array_equal(g[2].cpu().numpy(), ref.packed), (call, i, "packed vs oracle")
+            assert np.array_equal(g[3].cpu().view(torch.int16).numpy().view(np.uint16), ref.scale_f16), \
+                (call, i, "scale_f16 vs oracle")
 
 
 def test_noalloc_rejects_batches_beyond_its_scratch(gq):
