@@ -600,8 +600,80 @@ def measure_rows(gq, device, peak):
     batch([(s, wsu[s.name].view(np.int16)) for s in synth.unified11_train().specs], export=False,
           name="unified11 bf16 train step: fake-quant batched + STE", ste=True,
           note="cold L2; one iteration: w_hat (fp32 scales) of the 44 weights + STE copy of their gradients")
+    # GPTQ-lite export of the 11-layer d528 model: 44 bf16 weights, each
+    # against the binary64 Hessian of 2048 synthetic input rows of its own
+    gptq_rows(gq, device, out, record)
     torch.cuda.synchronize()
     return out
+
+
+FP64_FMA_PER_SM_CLK = 64       # B200: 64 binary64 FMA per SM per clock (CUDA cores)
+
+
+def fp64_peak_tflops(sm_mhz=None):
+    """Binary64 FMA peak derived from the SM count and clock: 148 SMs x 64 FMA
+    x 2 flops x clock (the measured SM clock when given, else 1965 MHz)."""
+    mhz = sm_mhz or 1965.0
+    return 148 * FP64_FMA_PER_SM_CLK * 2 * mhz * 1e6 / 1e12
+
+
+def gptq_rows(gq, device, out, record):
+    specs = synth.unified11_train().specs
+    wsu = synth.draw_unified11()
+    rng = np.random.default_rng(21)
+    items = []
+    for s in specs:
+        W = torch.from_numpy(wsu[s.name].view(np.int16).copy()).to(device).view(torch.bfloat16)
+        x = synth.gptq_calibration(rng, 2048, s.shape[1])
+        items.append((s, W, x, torch.from_numpy(x).to(device)))
+    Hs = [gq.gptq_hessian(X) for (_, _, _, X) in items]
+    reqs = [gq.Request(W, 6, 1.0, want_dq=False) for (_, W, _, _) in items]
+    # binary64 flops: the recurrence (rows * cols^2) and the Cholesky (cols^3 / 3)
+    fl = sum(s.shape[0] * s.shape[1] ** 2 + s.shape[1] ** 3 / 3.0 for (s, _, _, _) in items)
+    fl_h = sum(2 * 2048 * s.shape[1] ** 2 / 2 for (s, _, _, _) in items)
+
+    def run_all():
+        for r, H in zip(reqs, Hs):
+            gq.gptq_quantize(r, H, check_status=False)
+
+    def hess_all():
+        for (_, _, _, X), H in zip(items, Hs):
+            gq.gptq_hessian(X, H)
+
+    for name, fn, flops, note in (
+            ("gptq unified11 export (44 weights, int6 per row)", run_all, fl,
+             "binary64 recurrence + Cholesky, Hessians given; packed int6 + fp16 scales"),
+            ("gptq unified11 Hessians (2048 input rows each)", hess_all, fl_h, "H = 2 X^T X in binary64")):
+        t = statistics.median(_time_reps(fn, 5))
+        tf = flops / t / 1e12
+        out[name] = {"ms": round(t * 1e3, 3), "fp64_tflops": round(tf, 2),
+                     "alu_frac": round(tf / fp64_peak_tflops(), 3), "bound": "alu (binary64 FMA)",
+                     "peak_tflops": round(fp64_peak_tflops(), 1), "peak_source": "derived: 148 SM x 64 FMA x 2 x 1965 MHz",
+                     "note": note}
+    # CPU oracle on the first layer's four weights
+    from oracle import gptq as OG
+    t0 = time.perf_counter()
+    for (s, W, x, _) in items[:4]:
+        OG.gptq(wsu[s.name], OG.hessian(x), 6, 1.0)
+    cs = time.perf_counter() - t0
+    fl4 = sum(s.shape[0] * s.shape[1] ** 2 + s.shape[1] ** 3 / 3.0 for (s, _, _, _) in items[:4])
+    out["gptq unified11 export (44 weights, int6 per row)"]["cpu_oracle"] = {
+        "seconds": round(cs, 3), "fp64_gflops": round(fl4 / cs / 1e9, 3), "cores": 1, "kind": "oracle",
+        "sample": "the first layer's four weights (numpy binary64, LAPACK inverse and Cholesky)"}
+
+
+def _time_reps(fn, reps):
+    fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        b.synchronize()
+        ts.append(a.elapsed_time(b) / 1e3)
+    return ts
 
 
 def run_ours(args, world, rank, local):

@@ -25,6 +25,7 @@ namespace {
 using namespace gq;
 
 constexpr size_t kWsSlot = 8448;      // 2048 x u32 histogram + 16 x u32 state, 256-aligned
+constexpr int64_t kWaveBytes = 48ll << 20;   // per-tensor inputs per wave (L2 is 126 MB)
 constexpr int kMaxDevices = 64;
 std::atomic<int> g_sm_count[kMaxDevices];
 
@@ -372,6 +373,13 @@ gq_status quantize_batch(const gq_tensor* t, int n, Op op, bool f16_mode, void* 
     std::vector<RowDesc> rows_w, rows_c;   // warp teams / block teams
     std::vector<RowDesc> rows_tma;         // pipelined through shared memory
     std::vector<PassDesc> pass;
+    // per-tensor groups, in waves whose inputs fit in L2 together
+    struct Wave {
+        std::vector<SelDesc> sel;
+        std::vector<RowDesc> tma, w, c;
+        int64_t bytes = 0;
+    };
+    std::vector<Wave> waves;
     size_t slot = 0;
     for (int i = 0; i < n; ++i) {
         const gq_tensor& T = t[i];
@@ -454,17 +462,41 @@ gq_status quantize_batch(const gq_tensor* t, int n, Op op, bool f16_mode, void* 
             D.items = T.rows;
         }
         D.flags = flags;
+        std::vector<RowDesc>* tma = &rows_tma;
+        std::vector<RowDesc>* wt = &rows_w;
+        std::vector<RowDesc>* ct = &rows_c;
+        if (T.gran == GQ_PER_TENSOR) {
+            // a per-tensor group reads its tensor four times (three histogram
+            // passes, then the quantize pass): group the tensors in waves of
+            // at most kWaveBytes of input so that the later passes of a wave
+            // find its tensors in L2
+            const int64_t bytes = T.rows * T.cols * esz;
+            if (waves.empty() || (waves.back().bytes > 0 && waves.back().bytes + bytes > kWaveBytes))
+                waves.emplace_back();
+            Wave& Wv = waves.back();
+            Wv.bytes += bytes;
+            Wv.sel.push_back(sel.back());
+            sel.pop_back();
+            tma = &Wv.tma;
+            wt = &Wv.w;
+            ct = &Wv.c;
+        }
         // column scales read as float4 by the pipelined kernel (else the row kernels)
         if (tma_eligible(T, flags) && (!T.col_scale || (flags & kVecCol)))
-            rows_tma.push_back(D);
+            tma->push_back(D);
         else if (T.cols <= 2048)
-            rows_w.push_back(D);
+            wt->push_back(D);
         else
-            rows_c.push_back(D);
+            ct->push_back(D);
     }
 
-    gq_status st = run_per_tensor_select(sel, stream);
-    if (st != GQ_OK) return st;
+    gq_status st = GQ_OK;
+    for (Wave& Wv : waves) {
+        if ((st = run_per_tensor_select(Wv.sel, stream)) != GQ_OK) return st;
+        if ((st = run_rows_tma(Wv.tma, stream)) != GQ_OK) return st;
+        if ((st = run_rows<1>(Wv.w, stream)) != GQ_OK) return st;
+        if ((st = run_rows<kBlockWarps>(Wv.c, stream)) != GQ_OK) return st;
+    }
     st = run_rows_tma(rows_tma, stream);
     if (st != GQ_OK) return st;
     st = run_rows<1>(rows_w, stream);
@@ -491,25 +523,6 @@ PFN_cuTensorMapEncodeTiled encode_tiled() {
         g_encode_tiled.store(f, std::memory_order_release);
     }
     return reinterpret_cast<PFN_cuTensorMapEncodeTiled>(f);
-}
-
-// K splits for a grid of tiles_mn output tiles: the split count minimising
-// (waves of one-CTA-per-SM launches) x (per-CTA time), with a per-CTA cost
-// of about 5 us plus 0.15 us per 64-wide K stage (measured on the decode
-// shapes); each split keeps at least 8 stages.
-int gemm_splits(int64_t tiles_mn, int64_t k_stages) {
-    const double sms = (double)sm_count();
-    int best = 1;
-    double best_t = 1e30;
-    for (int64_t s = 1; s <= std::max<int64_t>(1, k_stages / 8) && s <= 64; ++s) {
-        const double waves = std::ceil((double)(tiles_mn * s) / sms);
-        const double t = waves * (5.0 + 0.15 * std::ceil((double)k_stages / (double)s));
-        if (t < best_t - 1e-9) {
-            best_t = t;
-            best = (int)s;
-        }
-    }
-    return best;
 }
 
 // Scratch of gq_export_pack_noalloc: a fixed device array that every call on
@@ -773,13 +786,16 @@ gq_status gq_gemm_dequant(const void* d_x, int64_t M, int64_t K, int64_t ldx, co
                           int32_t* d_status, cudaStream_t stream) {
     if (M < 0 || N < 0 || K < 0 || (qbits != 6 && qbits != 8)) return GQ_ERR_INVALID_ARG;
     if (ldx < K || ldy < N) return GQ_ERR_INVALID_ARG;
-    if (K % kGemmBK != 0 || M > INT32_MAX || K > INT32_MAX || N > INT32_MAX) return GQ_ERR_UNSUPPORTED;
+    if (M > INT32_MAX || K > INT32_MAX || N > INT32_MAX) return GQ_ERR_UNSUPPORTED;
+    const int64_t prb = packed_row_bytes(K, qbits);
+    const bool tma_codes = prb % 16 == 0;
+    if (!tma_codes && prb % 4 != 0) return GQ_ERR_UNSUPPORTED;   // int6 needs K % 16 == 0, int8 K % 4 == 0
     if (d_status && !aligned(d_status, 4)) return GQ_ERR_MISALIGNED;
     if (d_status && cuda_status(cudaMemsetAsync(d_status, 0, sizeof(int32_t), stream)) != GQ_OK) return GQ_ERR_CUDA;
     if (M == 0 || N == 0) return GQ_OK;
     if (!d_x || !d_packed || !d_scale_f16 || !d_y) return GQ_ERR_INVALID_ARG;
-    if (!aligned(d_x, 16) || (ldx % 8) != 0 || !aligned(d_packed, 16) || !aligned(d_scale_f16, 2) ||
-        !aligned(d_y, 16) || (ldy % 4) != 0)
+    if (!aligned(d_x, 16) || (ldx % 8) != 0 || !aligned(d_packed, tma_codes ? 16 : 4) ||
+        !aligned(d_scale_f16, 2) || !aligned(d_y, 4))
         return GQ_ERR_MISALIGNED;
     if (K == 0)
         return cuda_status(cudaMemset2DAsync(d_y, (size_t)ldy * 4, 0, (size_t)N * 4, (size_t)M, stream));
@@ -787,33 +803,49 @@ gq_status gq_gemm_dequant(const void* d_x, int64_t M, int64_t K, int64_t ldx, co
     if (!enc) return GQ_ERR_UNSUPPORTED;
     GemmParams P;
     std::memset(&P, 0, sizeof(P));
-    // a batch of at most 128 tokens swaps the operands: 128 weight rows x nt tokens
-    P.swap = M <= kGemmBM ? 1 : 0;
-    P.nt = kGemmBM;
-    if (P.swap) {
-        P.nt = 16;
-        while (P.nt < M) P.nt *= 2;
+    // token tile: the batch itself up to 256 tokens (rounded up to 16 .. 256), else 256
+    int nt = 16;
+    while (nt < M && nt < 256) nt *= 2;
+    P.nt = nt;
+    P.ni = nt <= 64 ? 2 : 1;
+    P.cs = nt <= 128 ? 4 : 2;                           // K stages per copy (an X chunk of at most 64 KB)
+    P.idesc = gemm_idesc(kGemmBN, (uint32_t)nt);
+    P.acc_cols = (uint32_t)std::max(32, nt);
+    const cuuint32_t estride[3] = {1, 1, 1};
+    // X: a 3-D view {64, M, K / 64} (one copy per chunk) when K % 64 == 0,
+    // else the 2-D [M, K] view (one copy per stage)
+    P.x3d = 0;
+    if (K % kGemmBK == 0) {
+        const cuuint64_t gdim3[3] = {(cuuint64_t)kGemmBK, (cuuint64_t)M, (cuuint64_t)(K / kGemmBK)};
+        const cuuint64_t gstride3[2] = {(cuuint64_t)ldx * 2, (cuuint64_t)kGemmBK * 2};
+        const cuuint32_t box3[3] = {(cuuint32_t)kGemmBK, (cuuint32_t)nt, (cuuint32_t)P.cs};
+        if (enc(&P.tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(d_x), gdim3, gstride3, box3, estride,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+            P.x3d = 1;
     }
-    P.idesc = gemm_idesc(kGemmBM, P.swap ? (uint32_t)P.nt : (uint32_t)kGemmBN);
-    P.acc_cols = P.swap ? (uint32_t)std::max(32, P.nt) : (uint32_t)kGemmBN;
-    P.tmem_cols = P.acc_cols * kGemmMmaWarps;
-    const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)M};
-    const cuuint64_t gstride[1] = {(cuuint64_t)ldx * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)kGemmBK, (cuuint32_t)P.nt};
-    const cuuint32_t estride[2] = {1, 1};
-    if (enc(&P.tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(d_x), gdim, gstride, box, estride,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return GQ_ERR_UNSUPPORTED;
-    const int64_t prb = packed_row_bytes(K, qbits);
-    const cuuint64_t wdim[2] = {(cuuint64_t)prb, (cuuint64_t)N};
-    const cuuint64_t wstride[1] = {(cuuint64_t)prb};
-    const int64_t stage_code_bytes = qbits == 6 ? 48 : 64;       // 64 codes of a row
-    const cuuint32_t wbox[2] = {(cuuint32_t)stage_code_bytes, (cuuint32_t)kGemmBN};
-    if (enc(&P.tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(d_packed), wdim, wstride, wbox,
-            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return GQ_ERR_UNSUPPORTED;
+    if (!P.x3d) {
+        const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)M};
+        const cuuint64_t gstride[1] = {(cuuint64_t)ldx * 2};
+        const cuuint32_t box[2] = {(cuuint32_t)kGemmBK, (cuuint32_t)nt};
+        if (enc(&P.tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(d_x), gdim, gstride, box, estride,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return GQ_ERR_UNSUPPORTED;
+    }
+    const int64_t cb = qbits == 6 ? 48 : 64;          // code bytes of a row's 64-code stage
+    const int64_t crow = cb * P.cs;                   // ... of a row's chunk
+    if (tma_codes) {
+        const cuuint64_t wdim[2] = {(cuuint64_t)prb, (cuuint64_t)N};
+        const cuuint64_t wstride[1] = {(cuuint64_t)prb};
+        const cuuint32_t wbox[2] = {(cuuint32_t)crow, (cuuint32_t)kGemmBN};
+        if (enc(&P.tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(d_packed), wdim, wstride, wbox,
+                estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return GQ_ERR_UNSUPPORTED;
+    }
+    P.code_copy = tma_codes ? 0 : 1;
+    P.codes = d_packed;
     P.scale = d_scale_f16;
     P.y = d_y;
     P.status = d_status;
@@ -821,28 +853,29 @@ gq_status gq_gemm_dequant(const void* d_x, int64_t M, int64_t K, int64_t ldx, co
     P.N = N;
     P.K = K;
     P.ldy = ldy;
+    P.prb = prb;
     P.qbits = qbits;
-    const int64_t tiles_n = (N + kGemmBN - 1) / kGemmBN, tiles_m = (M + P.nt - 1) / P.nt;
-    if (tiles_n > 0x7FFFFFFF || tiles_m > 65535) return GQ_ERR_UNSUPPORTED;
-    const int64_t k_stages = K / kGemmBK;
-    const int splits = gemm_splits(tiles_n * tiles_m, k_stages);
-    P.k_stages = (int32_t)k_stages;
-    P.splits = splits;
-    P.accumulate = splits > 1 ? 1 : 0;
-    // ring depths, all even: a waiter then always has seen the barrier's
-    // previous phase itself (stages alternate between two MMA warps and two
-    // dequant groups), so a parity test cannot be satisfied by a phase
-    // behind the one it waits for
-    const int64_t x_bytes = (int64_t)P.nt * 128;
-    const int64_t code_bytes = kGemmBN * stage_code_bytes;
-    // (the X ring covers a round trip X load -> dequant check -> MMA ->
-    // commit -> next X load of about 2 us; small token tiles take it deep)
-    P.w_stages = P.nt == 128 ? 4 : 6;
-    P.x_stages = P.nt <= 32 ? 14 : 8;
-    P.c_stages = (int32_t)std::min<int64_t>(
-        kGemmCStagesMax, (kGemmRingBytes - P.w_stages * (int64_t)kGemmAtomBytes - P.x_stages * x_bytes) / code_bytes);
-    P.c_stages &= ~1;
-    if (splits > 1 &&
+    P.kt_per_tile = (int32_t)((K + kGemmBK - 1) / kGemmBK);
+    const int64_t tiles_n = (N + kGemmBN - 1) / kGemmBN, tiles_m = (M + nt - 1) / nt;
+    P.tiles_m = (int32_t)tiles_m;
+    P.tiles = tiles_n * tiles_m;
+    const int64_t sms = sm_count();
+    // few tiles: split the stage units evenly (partial sums added into a
+    // zeroed Y); many: whole tiles round-robin
+    P.streamk = P.tiles < 2 * sms ? 1 : 0;
+    const int64_t units = P.streamk ? P.tiles * P.kt_per_tile : P.tiles;
+    const int64_t grid = std::min<int64_t>(sms, units);
+    // ring depths in chunks: X up to 64 KB (at least 2 slots), codes in what
+    // is left, W_hat in the TMEM columns after the accumulators; the commit
+    // ring is a multiple of the W_hat depth and at least the X depth (a
+    // waiter on any of these barriers then never sees a phase two ahead)
+    const int64_t x_bytes = (int64_t)nt * 128 * P.cs, c_bytes = kGemmBN * crow;
+    P.dx = (int32_t)std::max<int64_t>(2, std::min<int64_t>(8, (64 * 1024) / x_bytes));
+    P.dc = (int32_t)std::min<int64_t>(kGemmMaxC, (kGemmRingBytes - P.dx * x_bytes) / c_bytes);
+    P.dw = (int32_t)std::min<int64_t>(kGemmMaxW, (512 - P.ni * (int64_t)P.acc_cols) / (32 * P.cs));
+    P.dd = P.dw * ((P.dx + P.dw - 1) / P.dw);
+    if (P.dc < 2 || P.dw < 2 || P.dd > kGemmMaxDone || P.dx > kGemmMaxX) return GQ_ERR_UNSUPPORTED;
+    if (P.streamk &&
         cuda_status(cudaMemset2DAsync(d_y, (size_t)ldy * 4, 0, (size_t)N * 4, (size_t)M, stream)) != GQ_OK)
         return GQ_ERR_CUDA;
     int dev = 0;
@@ -853,8 +886,7 @@ gq_status gq_gemm_dequant(const void* d_x, int64_t M, int64_t K, int64_t ldx, co
             return GQ_ERR_CUDA;
         g_gemm_smem_set[dev].store(kGemmSmemBytes);
     }
-    const dim3 grid((unsigned)tiles_n, (unsigned)tiles_m, (unsigned)splits);
-    gemm_dequant_kernel<<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(P);
+    gemm_dequant_kernel<<<(unsigned)grid, kGemmThreads, kGemmSmemBytes, stream>>>(P);
     return launch_status();
 }
 

@@ -1,33 +1,54 @@
 // gq_gemm.cuh -- the consuming GEMM with the dequant fused into its weight
-// load: Y[M, N] (+)= X[M, K] * W_hat[N, K]^T on the 5th-generation tensor
-// cores, where W_hat[n, k] = bf16(RN(q[n, k] * s[n])) is rebuilt from the
-// packed int6 / int8 codes and binary16 row scales of an export while the
-// weight tile is staged in shared memory (the fake-quant weights of the
-// forward pass, "STE QAT" on "SubSixteen v2" and PR #1202, consumed where
-// the GEMM loads them instead of being written out and read back).
+// load: Y[M, N] = X[M, K] * W_hat[N, K]^T on the 5th-generation tensor cores,
+// where W_hat[n, k] = bf16(RN(q[n, k] * s[n])) is rebuilt from the packed
+// int6 / int8 codes and binary16 row scales of an export (the fake-quant
+// weights of the forward pass, "STE QAT" on "SubSixteen v2" and PR #1202,
+// consumed where the GEMM loads them instead of being written out and read
+// back).
 //
-// One CTA per output tile and K slice (split K for a small M).  For M > 128
-// the tile is 128 tokens x 128 weight rows (A = X, B = W_hat); for M <= 128
-// the operands swap (A = W_hat, 128 weight rows; B = X, nt = 16 .. 128 token
-// rows), so a small batch does not pay for 128-row MMAs on padding.
-//   warp 0        one lane loads the X tiles by TMA (SWIZZLE_128B, K-major)
-//   warp 1        one lane loads the packed code tiles by TMA, far ahead
-//   warps 2, 3    issue tcgen05.mma (kind::f16, bf16 x bf16 -> fp32, M 128,
-//                 K 16), stage kt by warp 2 + kt % 2 into accumulator kt % 2
-//   warps 4..19   dequantize, in two groups of 8 warps (stage kt by group
-//                 kt % 2, two threads per weight row), from the staged codes
-//                 into the SWIZZLE_128B K-major layout; then all 16 read the
-//                 accumulators out of TMEM (tcgen05.ld, four warps per lane
-//                 quarter), add them and store or add the sums into Y
-// A stage is one 64-wide swizzle atom of K (4 MMAs).  Every hand-off
-// between warps costs a few hundred ns of latency, so the work alternates
-// between two MMA warps and two dequant groups, and the rings (W_hat,
-// X and codes, each with its own depth) are deep enough that a slot's
-// round trip (dequant -> MMA -> commit -> dequant) overlaps the next
-// stages.  The MMA warp waits for the stage's X tile (TMA bytes) and
-// W_hat tile (the 256 arrivals of its dequant group); the stage's one
-// commit (on a ring of its own) frees both slots.  Every wait is bounded
-// by %globaltimer.
+// Tile: 128 weight rows x nt tokens (nt = 16 .. 256), K in stages of 64.
+// The operands are swapped so that the weight tile is the MMA's A operand
+// (M = 128) and the token tile its B operand (N = nt):
+//   - W_hat never touches shared memory: the dequant threads write it into
+//     tensor memory with tcgen05.st (thread r of a lane quarter owns weight
+//     row r of the tile), and tcgen05.mma reads A from there.  A 64-wide
+//     stage of W_hat is 32 TMEM columns (two bf16 per 32-bit column);
+//   - X tiles arrive by TMA (SWIZZLE_128B, K-major) in shared memory;
+//   - the packed codes arrive by TMA (or, for int6 rows whose byte length is
+//     not a multiple of 16, by 4-byte cp.async copies) in shared memory.
+// Shared memory then only carries codes and X, so the MMA's operand reads do
+// not compete with W_hat traffic, and an MMA of a small token tile runs at
+// about 40 ns per stage (four K = 16 MMAs) instead of ~120 ns with A staged in
+// shared memory.
+//
+// Persistent blocks, one per SM.  Work is a list of stage units (tile, k
+// stage), tile-major: with few tiles (decode-sized batches) the units are
+// split evenly over the blocks (stream-K: a block's range crosses tile
+// boundaries, every partial sum is added into Y, which is zeroed first);
+// otherwise each block takes whole tiles round-robin and stores them.
+//
+// Chunks.  One thread can start a TMA copy only about every 250 ns, whatever
+// its size, so copies move CS consecutive K stages at once (a chunk: CS = 4
+// for token tiles of up to 128, 2 for 256): one copy of the code rows
+// (128 rows x CS * 48 / 64 bytes) and one copy of the token tile (a 3-D
+// view of X, {64, nt, CS} with the 128-byte swizzle, when K % 64 == 0; else
+// one 2-D copy per stage).  A chunk is also the unit of the MMA hand-off:
+// one issuer runs all of a chunk's stages and commits once.  Chunks are
+// aligned to the tile's K stages; a block's first and last chunk of a tile
+// may hold only part of their stages (the copies still move the whole chunk).
+//
+// Warp roles (24 warps):
+//   warp 0        code producer (TMA, or 4-byte cp.async copies)
+//   warps 1, 2    MMA issuers: chunk c by issuer c % NI (NI = 2 for nt <= 64,
+//                 each with its own accumulator; else NI = 1)
+//   warp 3        TMEM allocation, then the X producer (TMA)
+//   warps 4 .. 7  epilogue: accumulators -> Y (one warp per lane quarter)
+//   warps 8 .. 23 dequant, four groups of four warps (one per lane quarter);
+//                 group g takes sub-stage g % CS of every (4 / CS)-th chunk
+// Every wait is an mbarrier wait bounded by %globaltimer; on expiry the
+// waiter records GQ_STATUS_TIMEOUT and its role stops.  Before the block
+// exits, the producers wait (bounded) for their copies in flight, the
+// issuers for their MMAs, and TMEM is released.
 #pragma once
 
 #include <cuda.h>
@@ -35,46 +56,43 @@
 
 namespace gq {
 
-constexpr int kGemmBM = 128;
-constexpr int kGemmBN = 128;
-constexpr int kGemmBK = 64;                              // a stage: one 128-byte swizzle atom of bf16 along K
-constexpr int kGemmWStagesMax = 8;                       // W_hat ring
-constexpr int kGemmXStagesMax = 14;                      // X ring
-constexpr int kGemmDoneRing = 32;                        // per-stage MMA commits (> twice either depth)
-constexpr int kGemmCStagesMax = 12;                      // code ring
-constexpr int kGemmMmaWarps = 2;                         // stage kt is issued by MMA warp kt % 2
-constexpr int kGemmDqGroups = 2;                         // stage kt is dequantized by group kt % 2
-constexpr int kGemmGroup = 2 * kGemmBN;                  // threads of a group: two per weight row
-constexpr int kGemmDequant = kGemmDqGroups * kGemmGroup;
-constexpr int kGemmDqWarp0 = 2 + kGemmMmaWarps;          // first dequant warp
-constexpr int kGemmThreads = 32 * kGemmDqWarp0 + kGemmDequant;
-constexpr int kGemmAtomBytes = kGemmBN * kGemmBK * 2;    // 16 KB: 128 rows x 64 bf16
-constexpr int kGemmBarBytes = 1024;
+constexpr int kGemmBN = 128;                             // weight rows per tile (the MMA's M)
+constexpr int kGemmBK = 64;                              // K per stage
+constexpr int kGemmGroups = 4;                           // dequant groups
+constexpr int kGemmCSMax = 4;                            // stages per chunk (max)
+constexpr int kGemmDq0 = 8;                              // first dequant warp
+constexpr int kGemmEpi0 = 4;                             // first epilogue warp
+constexpr int kGemmThreads = 32 * (kGemmDq0 + 4 * kGemmGroups);
+constexpr int kGemmMaxX = 16;                            // X chunk slots (max)
+constexpr int kGemmMaxC = 16;                            // code chunk slots (max)
+constexpr int kGemmMaxW = 4;                             // W_hat chunk slots in TMEM (max)
+constexpr int kGemmMaxDone = 32;                         // per-chunk MMA commit ring (max)
+constexpr int kGemmBarBytes = 8 * (kGemmMaxX + 2 * kGemmMaxC + kGemmMaxW * kGemmCSMax + kGemmMaxDone + 8) + 64;
 constexpr int kGemmSmemBytes = 232448;                   // all of it: 227 KB
 constexpr int kGemmRingBytes = kGemmSmemBytes - 1024 /* alignment */ - kGemmBarBytes;
 constexpr unsigned long long kGemmWaitNs = 4000000000ull;
-static_assert(kGemmDoneRing % kGemmMmaWarps == 0 && kGemmDoneRing % kGemmDqGroups == 0, "commit ring");
-static_assert(2 * kGemmWStagesMax < kGemmDoneRing && 2 * kGemmXStagesMax < kGemmDoneRing, "commit ring depth");
 
 struct GemmParams {
-    CUtensorMap tmap_x;          // X [M, K] bf16, box 64 x nt, SWIZZLE_128B
-    CUtensorMap tmap_w;          // codes [N, prb] bytes, box (64 codes' bytes) x 128, no swizzle
+    CUtensorMap tmap_x;          // X: 3-D {64, M, K / 64} box {64, nt, CS}, or 2-D [M, K] box {64, nt}; SWIZZLE_128B
+    CUtensorMap tmap_w;          // codes [N, prb] bytes, box (CS stages' bytes) x 128, no swizzle (TMA mode)
+    const uint8_t* codes;        // packed codes (copy mode)
     const uint16_t* scale;       // [N] binary16 row scales
-    float* y;                    // [M, ldy] fp32, added into (split K) or stored
+    float* y;                    // [M, ldy] fp32
     int32_t* status;             // nullable: GQ_STATUS_TIMEOUT on an expired wait
-    int64_t M, N, K, ldy;
+    int64_t M, N, K, ldy, prb;
     int32_t qbits;
-    int32_t k_stages;            // 64-wide K stages in all
-    int32_t splits;              // K splits (grid z); split z takes a contiguous run of stages
-    int32_t accumulate;          // 1: red.add into Y (split K), 0: store
-    int32_t swap;                // 1: A = W_hat, B = X (M <= 128)
-    int32_t nt;                  // token rows of an X tile (128, or 16 .. 128 swapped)
-    uint32_t idesc;              // tcgen05 instruction descriptor of the tile's MMA
-    uint32_t tmem_cols;          // TMEM columns allocated: kGemmMmaWarps accumulators
-    uint32_t acc_cols;           // columns of one accumulator (a power of two >= 32)
-    int32_t w_stages;            // ring depths
-    int32_t x_stages;
-    int32_t c_stages;
+    int32_t code_copy;           // 1: codes by cp.async (prb % 16 != 0), 0: by TMA
+    int32_t x3d;                 // 1: one 3-D copy of X per chunk, 0: one 2-D copy per stage
+    int32_t cs;                  // stages per chunk
+    int32_t kt_per_tile;         // 64-wide K stages per tile
+    int32_t tiles_m;             // token tiles
+    int64_t tiles;               // tiles_n * tiles_m
+    int32_t streamk;             // 1: stage units split evenly, partial sums added; 0: whole tiles
+    int32_t nt;                  // tokens per tile (the MMA's N)
+    int32_t ni;                  // MMA issuers (accumulators)
+    uint32_t idesc;              // tcgen05 instruction descriptor
+    uint32_t acc_cols;           // TMEM columns of one accumulator
+    int32_t dx, dc, dw, dd;      // ring depths in chunks: X, codes, W_hat (TMEM), MMA commits
 };
 
 // ------------------------------------------------------------- PTX glue --
@@ -89,17 +107,14 @@ __device__ __forceinline__ unsigned long long g_now() {
     return t;
 }
 
-// Test for the completion of the phase with the given parity; the thread
-// may sleep in the barrier for up to the hint (100 us) while it waits, so
-// that waiting warps leave the issue slots to the working ones.
 __device__ __forceinline__ bool g_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t done;
     asm volatile(
         "{\n .reg .pred p;\n"
-        " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+        " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
         " selp.u32 %0, 1, 0, p;\n}"
         : "=r"(done)
-        : "r"(bar), "r"(parity), "r"(100000u)
+        : "r"(bar), "r"(parity)
         : "memory");
     return done != 0;
 }
@@ -108,10 +123,15 @@ __device__ __forceinline__ bool g_try_wait(uint32_t bar, uint32_t parity) {
 __device__ __forceinline__ bool g_wait(uint32_t bar, uint32_t parity) {
     if (g_try_wait(bar, parity)) return true;
     const unsigned long long t0 = g_now();
-    for (;;) {
+    for (uint32_t i = 1;; ++i) {
         if (g_try_wait(bar, parity)) return true;
-        if (g_now() - t0 > kGemmWaitNs) return false;
+        if ((i & 63u) == 0u && g_now() - t0 > kGemmWaitNs) return false;
     }
+}
+
+// g_wait by every lane of a warp, with a warp-uniform result.
+__device__ __forceinline__ bool g_wait_warp(uint32_t bar, uint32_t parity) {
+    return __all_sync(0xffffffffu, g_wait(bar, parity));
 }
 
 __device__ __forceinline__ void g_bar_init(uint32_t bar, uint32_t count) {
@@ -135,6 +155,32 @@ __device__ __forceinline__ void g_tma_load_2d(uint32_t dst, const CUtensorMap* m
         : "memory");
 }
 
+// 3-D tiled TMA load (no multicast) of box {x, y, z} into this CTA's shared memory.
+__device__ __forceinline__ void g_tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
+                                              uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+        : "memory");
+}
+
+// `count` arrivals on `bar` at once.
+__device__ __forceinline__ void g_arrive_n(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+// 4-byte asynchronous copy global -> shared; `src_bytes` 0 fills zeros.
+__device__ __forceinline__ void g_cp_async4(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+
+// Arrive on `bar` once this thread's earlier cp.async copies have landed
+// (the barrier's expected count includes this arrival).
+__device__ __forceinline__ void g_cp_async_arrive(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+
 // Shared-memory matrix descriptor: K-major, SWIZZLE_128B, 8-row groups
 // 1024 bytes apart (stride byte offset), leading byte offset 16 (unused by
 // the swizzled K-major form), descriptor version 1.
@@ -149,45 +195,27 @@ __host__ __device__ constexpr uint32_t gemm_idesc(uint32_t m, uint32_t n) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((n >> 3) << 17) | ((m >> 4) << 24);
 }
 
-// One elected lane of a converged warp.
-__device__ __forceinline__ bool g_elect() {
-    uint32_t e;
-    asm volatile(
-        "{\n .reg .pred e;\n"
-        " elect.sync _|e, 0xffffffff;\n"
-        " selp.u32 %0, 1, 0, e;\n}"
-        : "=r"(e));
-    return e != 0;
-}
-
-// g_wait by every lane of a warp, with a warp-uniform result.
-__device__ __forceinline__ bool g_wait_warp(uint32_t bar, uint32_t parity) {
-    return __all_sync(0xffffffffu, g_wait(bar, parity));
-}
-
-// The 4 MMAs (K = 16 each) of one stage, issued by one elected lane of
-// the (converged) calling warp from a single asm block: nothing runs
-// between them in the issuing thread, which keeps the tensor pipe fed
-// (scalar work between consecutive tcgen05.mma roughly halves the issue
-// rate).  The first MMA into an accumulator overwrites it (accumulate = 0).
-__device__ __forceinline__ void g_mma_stage(uint32_t tmem, const uint64_t (&a)[4], const uint64_t (&b)[4],
-                                            uint32_t idesc, uint32_t accumulate) {
+// The 4 MMAs (K = 16 each) of one stage, A from tensor memory (8 columns
+// per K = 16 step), B from shared memory (32 bytes per step inside the
+// swizzle atom), issued by one elected lane from a single asm block.
+__device__ __forceinline__ void g_mma_stage_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_addr, uint32_t idesc,
+                                               uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p, e;\n\t"
         "setp.ne.b32 p, %9, 0;\n\t"
         "elect.sync _|e, 0xffffffff;\n\t"
-        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %5, %10, p;\n\t"
-        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %6, %10, 1;\n\t"
-        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %7, %10, 1;\n\t"
-        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %8, %10, 1;\n\t"
-        "}\n" ::"r"(tmem),
-        "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "r"(accumulate),
-        "r"(idesc)
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %5, %10, p;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], %6, %10, 1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %7, %10, 1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %8, %10, 1;\n\t"
+        "}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "r"(a_tmem + 8u), "r"(a_tmem + 16u), "r"(a_tmem + 24u), "l"(g_smem_desc(b_addr)),
+        "l"(g_smem_desc(b_addr + 32u)), "l"(g_smem_desc(b_addr + 64u)), "l"(g_smem_desc(b_addr + 96u)),
+        "r"(accumulate), "r"(idesc)
         : "memory");
 }
 
-// Arrive on `bar` once every tcgen05 operation issued so far is done (one
-// elected lane of the calling warp commits).
+// Arrive on `bar` once every tcgen05 operation this thread issued is done.
 __device__ __forceinline__ void g_commit(uint32_t bar) {
     asm volatile(
         "{\n\t.reg .pred e;\n\t"
@@ -196,21 +224,26 @@ __device__ __forceinline__ void g_commit(uint32_t bar) {
         : "memory");
 }
 
-// 16 consecutive accumulator columns of this thread's TMEM lane, summed
-// over the `nacc` accumulators `stride` columns apart (in accumulator order).
-__device__ __forceinline__ void g_acc16(uint32_t taddr, uint32_t stride, int nacc, float (&f)[16]) {
-    for (int a = 0; a < nacc; ++a) {
-        uint32_t v[16];
-        asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
-            "%12, %13, %14, %15}, [%16];"
-            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-              "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
-            : "r"(taddr + (uint32_t)a * stride));
-        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+__device__ __forceinline__ void g_tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
+}
+
+__device__ __forceinline__ void g_tmem_ld16(uint32_t taddr, float (&f)[16]) {
+    uint32_t v[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+        "%12, %13, %14, %15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-        for (int i = 0; i < 16; ++i) f[i] = a == 0 ? __uint_as_float(v[i]) : __fadd_rn(f[i], __uint_as_float(v[i]));
-    }
+    for (int i = 0; i < 16; ++i) f[i] = __uint_as_float(v[i]);
 }
 
 // ------------------------------------------------------------- dequant --
@@ -276,74 +309,142 @@ __device__ __forceinline__ uint32_t g_pair_bf16(float f0, float f1, uint64_t s2,
     return g_bf16x2(w0, w1);
 }
 
-// Half a stage of one weight row: 32 codes (half of the swizzle atom,
-// chunks 4h .. 4h + 3) staged at `codes` (the code stage is released on
-// `release` once they are used), as bf16(RN(q * s)) into the K-major
-// SWIZZLE_128B layout (16-byte chunk c of row r at chunk position c ^ (r & 7)
-// of the row's 128 bytes at `row_addr`).
+// Codes 2i and 2i + 1 of a 64-code stage held in w[] (int6: 12 words and a
+// zero; int8: 16 words) as one bf16x2 word of W_hat.
 template <int QBITS>
-__device__ __forceinline__ void g_dequant_part(uint32_t codes, uint32_t release, uint32_t row_addr, int r, int h,
-                                               const GDeq& d) {
-    uint32_t w[8];                                         // int6: 6 words (+1 zero); int8: 8 words
+__device__ __forceinline__ uint32_t g_pair(const uint32_t (&w)[16], int i, const GDeq& d) {
+    if constexpr (QBITS == 6) {
+        // the code stream shifted right by 12 (i - 1) holds code 2i at bit
+        // 12; shifted by 12 i it holds code 2i + 1 at bit 6
+        const int sh = 12 * i;
+        const uint32_t vb = __funnelshift_r(w[sh >> 5], w[(sh >> 5) + 1], sh & 31);
+        uint32_t va;
+        if (i == 0) {
+            va = w[0] << 12;
+        } else {
+            const int sa = sh - 12;
+            va = __funnelshift_r(w[sa >> 5], w[(sa >> 5) + 1], sa & 31);
+        }
+        return g_pair_bf16(g_field(va, 0x3F000u, 0x4B020000u), g_field(vb, 0xFC0u, 0x4B000800u), d.s_a, d.c_a);
+    } else {
+        const uint32_t wd = w[i >> 1];
+        if ((i & 1) == 0)                                  // bytes 0, 1: both at bit 8
+            return g_pair_bf16(g_field(wd << 8, 0xFF00u, 0x4B008000u), g_field(wd, 0xFF00u, 0x4B008000u), d.s_a,
+                               d.c_a);
+        const uint32_t v = wd >> 12;                       // bytes 2, 3: at bits 4 and 12 of wd >> 12
+        return g_pair_bf16(g_field(v, 0xFF0u, 0x4B000800u), g_field(v, 0xFF000u, 0x4B080000u), d.s_b, d.c_b);
+    }
+}
+
+// One weight row's 64-code stage (at shared address `codes`) into the 32
+// TMEM columns at `taddr` of this thread's lane.
+template <int QBITS>
+__device__ __forceinline__ void g_dequant_stage(uint32_t codes, uint32_t taddr, const GDeq& d) {
+    uint32_t w[16];
     if constexpr (QBITS == 6) {
 #pragma unroll
-        for (int i = 0; i < 3; ++i)                        // 24 bytes, 8-byte aligned
-            asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];"
-                         : "=r"(w[2 * i]), "=r"(w[2 * i + 1])
-                         : "r"(codes + 8u * i)
+        for (int i = 0; i < 3; ++i)                        // 48 bytes, 16-byte aligned
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(w[4 * i]), "=r"(w[4 * i + 1]), "=r"(w[4 * i + 2]), "=r"(w[4 * i + 3])
+                         : "r"(codes + 16u * i)
                          : "memory");
-        w[6] = 0u;
+        w[12] = w[13] = w[14] = w[15] = 0u;
     } else {
 #pragma unroll
-        for (int i = 0; i < 2; ++i)
+        for (int i = 0; i < 4; ++i)
             asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                          : "=r"(w[4 * i]), "=r"(w[4 * i + 1]), "=r"(w[4 * i + 2]), "=r"(w[4 * i + 3])
                          : "r"(codes + 16u * i)
                          : "memory");
     }
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {                          // 4 chunks of 8 codes
-        uint32_t out[4];
+    for (int h = 0; h < 2; ++h) {
+        uint32_t out[16];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int i = 4 * c + j;                       // codes 2i and 2i + 1
-            if constexpr (QBITS == 6) {
-                // the code stream shifted right by 12 (i - 1) holds code 2i at
-                // bit 12; shifted by 12 i it holds code 2i + 1 at bit 6
-                const int sh = 12 * i;
-                const uint32_t vb = __funnelshift_r(w[sh >> 5], w[(sh >> 5) + 1], sh & 31);
-                uint32_t va;
-                if (i == 0) {
-                    va = w[0] << 12;
-                } else {
-                    const int sa = sh - 12;
-                    va = __funnelshift_r(w[sa >> 5], w[(sa >> 5) + 1], sa & 31);
-                }
-                out[j] = g_pair_bf16(g_field(va, 0x3F000u, 0x4B020000u), g_field(vb, 0xFC0u, 0x4B000800u), d.s_a,
-                                     d.c_a);
-            } else {
-                const uint32_t wd = w[i >> 1];
-                if ((i & 1) == 0) {                        // bytes 0, 1: both at bit 8
-                    out[j] = g_pair_bf16(g_field(wd << 8, 0xFF00u, 0x4B008000u), g_field(wd, 0xFF00u, 0x4B008000u),
-                                         d.s_a, d.c_a);
-                } else {                                   // bytes 2, 3: at bits 4 and 12 of wd >> 12
-                    const uint32_t v = wd >> 12;
-                    out[j] = g_pair_bf16(g_field(v, 0xFF0u, 0x4B000800u), g_field(v, 0xFF000u, 0x4B080000u), d.s_b,
-                                         d.c_b);
-                }
-            }
-        }
-        const uint32_t dst = row_addr + (uint32_t)(((4 * h + c) ^ (r & 7)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(out[0]), "r"(out[1]), "r"(out[2]),
-                     "r"(out[3])
-                     : "memory");
+        for (int j = 0; j < 16; ++j) out[j] = g_pair<QBITS>(w, 16 * h + j, d);
+        g_tmem_st16(taddr + 16u * (uint32_t)h, out);
     }
-    // The code slot is released only now that every loaded word has been
-    // used: an arrive issued while a shared load is still in flight lets the
-    // next TMA copy (async proxy) overwrite the slot before the load reads
-    // it, and the release order of the arrive does not cover that.
-    g_arrive(release);
 }
+
+// -------------------------------------------------------- chunk schedule --
+
+// The block's chunks in order, walked incrementally (no division in the
+// loops: a 64-bit division costs far more than a hand-off).  The block owns
+// the stage units [u0, u1) (stream-K, tile-major) or whole tiles blockIdx.x,
+// blockIdx.x + gridDim.x, ...; a chunk is the part of one aligned run of CS
+// K stages of one tile that the block owns: sub-stages lo .. hi.  A segment
+// is a run of the block's chunks of one tile.
+struct CIter {
+    int64_t tile, step;
+    int64_t rem;                 // stages of the block not yet walked
+    int64_t seq;                 // chunk index within the block
+    int kt, KT, CS;
+    int c, lo, hi;               // the chunk: index within the tile, first and last owned sub-stage
+    bool seg_first, seg_last, seg_full;
+    int seg_kt0;
+    __device__ __forceinline__ void set() {
+        c = kt / CS;                                       // 32-bit: cheap
+        lo = kt - c * CS;
+        const int chunk_end = min(CS - 1, KT - 1 - c * CS);
+        hi = (int)min((int64_t)chunk_end, (int64_t)lo + rem - 1);
+        seg_first = kt == 0 || seq == 0;
+        if (seg_first) seg_kt0 = kt;
+        const int kt_last = c * CS + hi;
+        seg_last = kt_last == KT - 1 || rem == (int64_t)(hi - lo + 1);
+        seg_full = seg_kt0 == 0 && kt_last == KT - 1;
+    }
+    __device__ __forceinline__ void init(const GemmParams& P) {
+        KT = P.kt_per_tile;
+        CS = P.cs;
+        seq = 0;
+        if (P.streamk) {
+            const int64_t total = P.tiles * (int64_t)KT;
+            const int64_t u0 = total * (int64_t)blockIdx.x / gridDim.x;
+            const int64_t u1 = total * ((int64_t)blockIdx.x + 1) / gridDim.x;
+            rem = u1 - u0;
+            tile = u0 / KT;
+            kt = (int)(u0 - tile * KT);
+            step = 1;
+        } else {
+            const int64_t my = P.tiles > (int64_t)blockIdx.x ? (P.tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+            rem = my * KT;
+            tile = blockIdx.x;
+            kt = 0;
+            step = gridDim.x;
+        }
+        seg_kt0 = kt;
+        if (rem > 0) set();
+    }
+    __device__ __forceinline__ bool valid() const { return rem > 0; }
+    __device__ __forceinline__ void next() {
+        const int n = hi - lo + 1;
+        rem -= n;
+        kt += n;
+        if (kt == KT) {
+            kt = 0;
+            tile += step;
+        }
+        ++seq;
+        if (rem > 0) set();
+    }
+};
+
+// Slot and phase of a ring of D barriers or buffers, advanced one use at a time.
+struct GRing {
+    int s, D;
+    uint32_t ph;
+    __device__ __forceinline__ void init(int depth) {
+        s = 0;
+        D = depth;
+        ph = 0u;
+    }
+    __device__ __forceinline__ void next() {
+        if (++s == D) {
+            s = 0;
+            ph ^= 1u;
+        }
+    }
+};
 
 // ----------------------------------------------------------------- kernel --
 
@@ -351,52 +452,58 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_dequant_kernel(const __g
     extern __shared__ unsigned char g_smem[];
     const uint32_t raw = g_smem_u32(g_smem);
     const uint32_t base = (raw + 1023u) & ~1023u;          // SWIZZLE_128B tiles: 1024-byte aligned
-    // [W_hat ring][X ring][code ring: 128 rows x 48 | 64 bytes][barriers]
-    const int DW = P.w_stages, DX = P.x_stages, DC = P.c_stages;
-    const uint32_t x_bytes = (uint32_t)P.nt * 128u;
-    const uint32_t row_code_bytes = P.qbits == 6 ? 48u : 64u;        // 64 codes of a row
-    const uint32_t xs0 = base + (uint32_t)DW * kGemmAtomBytes;
-    const uint32_t cs0 = xs0 + (uint32_t)DX * x_bytes;
+    const int DX = P.dx, DC = P.dc, DW = P.dw, DD = P.dd, NT = P.nt, NI = P.ni, CS = P.cs;
+    const uint32_t xs_bytes = (uint32_t)NT * 128u;         // one stage of X
+    const uint32_t x_bytes = xs_bytes * (uint32_t)CS;      // an X chunk slot
+    const uint32_t cb = P.qbits == 6 ? 48u : 64u;          // code bytes of a row's 64-code stage
+    const uint32_t crow = cb * (uint32_t)CS;               // code bytes of a row's chunk
+    const uint32_t c_bytes = (uint32_t)kGemmBN * crow;     // a code chunk slot
+    // [X ring][code ring][barriers]
+    const uint32_t cs0 = base + (uint32_t)DX * x_bytes;
     const uint32_t bars = base + (uint32_t)(kGemmSmemBytes - 1024 - kGemmBarBytes);
-    auto full_w = [&](int s) { return bars + 8u * (uint32_t)s; };                      // a group's arrivals
-    auto full_x = [&](int s) { return bars + 8u * (uint32_t)(kGemmWStagesMax + s); };  // X TMA bytes
-    auto mma_done = [&](int kt) {                                                      // stage kt's commit
-        return bars + 8u * (uint32_t)(kGemmWStagesMax + kGemmXStagesMax + kt % kGemmDoneRing);
+    auto full_x = [&](int s) { return bars + 8u * (uint32_t)s; };
+    auto full_c = [&](int s) { return bars + 8u * (uint32_t)(kGemmMaxX + s); };
+    auto empty_c = [&](int s) { return bars + 8u * (uint32_t)(kGemmMaxX + kGemmMaxC + s); };
+    auto full_w = [&](int s, int k) {                      // sub-stage k of W_hat chunk slot s
+        return bars + 8u * (uint32_t)(kGemmMaxX + 2 * kGemmMaxC + s * kGemmCSMax + k);
     };
-    constexpr int kCBar = kGemmWStagesMax + kGemmXStagesMax + kGemmDoneRing;
-    auto full_c = [&](int s) { return bars + 8u * (uint32_t)(kCBar + s); };
-    auto empty_c = [&](int s) { return bars + 8u * (uint32_t)(kCBar + kGemmCStagesMax + s); };
-    const uint32_t done = bars + 8u * (uint32_t)(kCBar + 2 * kGemmCStagesMax);
-    const uint32_t tmem_slot = done + 8u;
-    auto w_tile = [&](int s) { return base + (uint32_t)s * kGemmAtomBytes; };
-    auto x_tile = [&](int s) { return xs0 + (uint32_t)s * x_bytes; };
-    auto c_tile = [&](int s) { return cs0 + (uint32_t)s * (kGemmBN * row_code_bytes); };
-    // parity of stage kt's commit on its done barrier
-    auto done_parity = [&](int kt) { return (uint32_t)((kt / kGemmDoneRing) & 1); };
+    auto done = [&](int s) {                               // a chunk's MMA commit
+        return bars + 8u * (uint32_t)(kGemmMaxX + 2 * kGemmMaxC + kGemmMaxW * kGemmCSMax + s);
+    };
+    const uint32_t acc_full0 =
+        bars + 8u * (uint32_t)(kGemmMaxX + 2 * kGemmMaxC + kGemmMaxW * kGemmCSMax + kGemmMaxDone);
+    auto acc_full = [&](int j) { return acc_full0 + 8u * (uint32_t)j; };   // issuer j's segment sums are ready
+    const uint32_t acc_empty = acc_full0 + 16u;                             // the epilogue has read them
+    const uint32_t fin = acc_full0 + 24u;                                   // 2 barriers: an issuer's MMAs are all done
+    const uint32_t tmem_slot = acc_full0 + 40u;
+    auto x_tile = [&](int s) { return base + (uint32_t)s * x_bytes; };
+    auto c_tile = [&](int s) { return cs0 + (uint32_t)s * c_bytes; };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t n0 = (int64_t)blockIdx.x * kGemmBN;
-    const int64_t m0 = (int64_t)blockIdx.y * P.nt;
-    const int kbase = P.k_stages / P.splits, kextra = P.k_stages % P.splits;
-    const int KT = kbase + ((int)blockIdx.z < kextra ? 1 : 0);
-    const int kt0 = (int)blockIdx.z * kbase + min((int)blockIdx.z, kextra);
+    CIter it;
+    it.init(P);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < DW; ++s) g_bar_init(full_w(s), kGemmGroup);
         for (int s = 0; s < DX; ++s) g_bar_init(full_x(s), 1);
-        for (int s = 0; s < kGemmDoneRing; ++s) g_bar_init(mma_done(s), 1);
         for (int s = 0; s < DC; ++s) {
-            g_bar_init(full_c(s), 1);
-            g_bar_init(empty_c(s), kGemmGroup);
+            g_bar_init(full_c(s), P.code_copy ? 32 : 1);
+            g_bar_init(empty_c(s), 4 * CS);                // four warps per sub-stage
         }
-        g_bar_init(done, kGemmMmaWarps);
+        for (int s = 0; s < DW; ++s)
+            for (int k = 0; k < CS; ++k) g_bar_init(full_w(s, k), 4);
+        for (int s = 0; s < DD; ++s) g_bar_init(done(s), 1);
+        g_bar_init(acc_full(0), 1);
+        g_bar_init(acc_full(1), 1);
+        g_bar_init(acc_empty, 4);                          // the four epilogue warps
+        g_bar_init(fin, 1);
+        g_bar_init(fin + 8u, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        if (!P.code_copy)
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&P.tmap_w)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&P.tmap_x)) : "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&P.tmap_w)) : "memory");
     }
-    if (warp == 2) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(tmem_slot),
-                     "r"(P.tmem_cols)
+    if (warp == 3) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(tmem_slot)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
@@ -405,164 +512,245 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_dequant_kernel(const __g
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     uint32_t tmem;
     asm volatile("ld.shared.b32 %0, [%1];" : "=r"(tmem) : "r"(tmem_slot) : "memory");
+    const uint32_t w_col0 = (uint32_t)NI * P.acc_cols;     // W_hat chunk slots after the accumulators
 
     bool ok = true;
-    // The control warps run their loops with all 32 lanes (the waits and
-    // the descriptor arithmetic stay warp-uniform); one elected lane issues
-    // each copy, MMA and commit.
-    const bool leader = g_elect();
     if (warp == 0) {
-        // ------------------------------------------------ X tiles (TMA) --
-        int issued = 0;
-        for (int kt = 0; kt < KT && ok; ++kt) {
-            const int s = kt % DX;
-            // the slot's previous stage has been consumed by its MMAs
-            if (kt >= DX && !g_wait_warp(mma_done(kt - DX), done_parity(kt - DX))) ok = false;
-            if (!ok) break;
-            if (leader) {
-                g_arrive_tx(full_x(s), x_bytes);
-                g_tma_load_2d(x_tile(s), &P.tmap_x, (kt0 + kt) * kGemmBK, (int)m0, full_x(s));
+        // ------------------------------------------------ code producer --
+        GRing rc;
+        rc.init(DC);
+        int64_t cur_tile = -1;
+        int n0 = 0;
+        int64_t issued = 0;
+        for (; it.valid() && ok; it.next(), rc.next()) {
+            if (it.tile != cur_tile) {
+                cur_tile = it.tile;
+                n0 = (int)(it.tile / P.tiles_m) * kGemmBN;
             }
-            issued = kt + 1;
-        }
-        // no copy may still be landing when the CTA leaves (instant unless a wait expired)
-        for (int kt = max(0, issued - DX); kt < issued; ++kt)
-            if (!g_wait_warp(full_x(kt % DX), (uint32_t)((kt / DX) & 1))) ok = false;
-    } else if (warp == 1) {
-        // --------------------------------------------- code tiles (TMA) --
-        int issued = 0;
-        for (int kt = 0; kt < KT && ok; ++kt) {
-            const int s = kt % DC, g = kt / DC;
-            if (g > 0 && !g_wait_warp(empty_c(s), (uint32_t)((g - 1) & 1))) ok = false;
-            if (!ok) break;
-            if (leader) {
-                g_arrive_tx(full_c(s), kGemmBN * row_code_bytes);   // out-of-range rows are zero-filled
-                g_tma_load_2d(c_tile(s), &P.tmap_w, (kt0 + kt) * (int)row_code_bytes, (int)n0, full_c(s));
+            // the slot's previous chunk has been read by its dequant warps
+            if (it.seq >= DC && !g_wait_warp(empty_c(rc.s), rc.ph ^ 1u)) {
+                ok = false;
+                break;
             }
-            issued = kt + 1;
+            if (!P.code_copy) {
+                if (lane == 0) {
+                    g_arrive_tx(full_c(rc.s), c_bytes);    // out-of-range rows / bytes are zero-filled
+                    g_tma_load_2d(c_tile(rc.s), &P.tmap_w, it.c * (int)crow, n0, full_c(rc.s));
+                }
+            } else {
+                // 4-byte copies of every row's chunk bytes; past the row end
+                // and past the last weight row zeros are filled in
+                const uint32_t words = crow / 4u;
+                const int64_t off0 = (int64_t)it.c * crow;
+                for (uint32_t e = (uint32_t)lane; e < (uint32_t)kGemmBN * words; e += 32u) {
+                    const uint32_t r = e / words, wi = e - r * words;
+                    const int64_t n = n0 + r;
+                    const int64_t off = off0 + 4 * wi;
+                    const bool in = n < P.N && off + 4 <= P.prb;
+                    const uint8_t* src = in ? P.codes + n * P.prb + off : P.codes;
+                    g_cp_async4(c_tile(rc.s) + r * crow + 4u * wi, src, in ? 4u : 0u);
+                }
+                g_cp_async_arrive(full_c(rc.s));
+            }
+            // sub-stages the block does not own are released here, so that the
+            // slot's release count is always four warps per sub-stage
+            const int missing = CS - (it.hi - it.lo + 1);
+            if (lane == 0 && missing > 0) g_arrive_n(empty_c(rc.s), 4u * (uint32_t)missing);
+            issued = it.seq + 1;
         }
-        for (int kt = max(0, issued - DC); kt < issued; ++kt)
-            if (!g_wait_warp(full_c(kt % DC), (uint32_t)((kt / DC) & 1))) ok = false;
-    } else if (warp < kGemmDqWarp0) {
-        // ------------------------------------------------------- MMA --
-        // MMA warp j issues stages j, j + 2, ... into accumulator j: the
-        // issuing thread's serial latency (barrier wait, descriptors,
-        // commit) is shared between the warps, and the tensor pipe takes
-        // their MMAs as they come
-        const int j = warp - 2;
-        const uint32_t acc = tmem + (uint32_t)j * P.acc_cols;
-        for (int kt = j; kt < KT && ok; kt += kGemmMmaWarps) {
-            const int s = kt % DW, sx = kt % DX;
-            // the stage's X tile (TMA) and W_hat tile (dequant) are in place
-            if (!g_wait_warp(full_x(sx), (uint32_t)((kt / DX) & 1)) ||
-                !g_wait_warp(full_w(s), (uint32_t)((kt / DW) & 1))) {
+        // no copy may still be landing when the block exits
+        for (int64_t q = max((int64_t)0, issued - DC); q < issued; ++q)
+            if (!g_wait_warp(full_c((int)(q % DC)), (uint32_t)((q / DC) & 1))) ok = false;
+    } else if (warp == 3) {
+        // --------------------------------------------------- X producer --
+        GRing rx, rdx;                                     // X slots, the commit of chunk seq - DX
+        rx.init(DX);
+        rdx.init(DD);
+        int64_t cur_tile = -1;
+        int m0 = 0;
+        int64_t issued = 0;
+        for (; it.valid() && ok; it.next(), rx.next()) {
+            if (it.tile != cur_tile) {
+                cur_tile = it.tile;
+                m0 = (int)(it.tile % P.tiles_m) * NT;
+            }
+            // the slot's previous chunk has been consumed by its MMAs
+            if (it.seq >= DX) {
+                if (!g_wait_warp(done(rdx.s), rdx.ph)) {
+                    ok = false;
+                    break;
+                }
+                rdx.next();
+            }
+            if (lane == 0) {
+                if (P.x3d) {
+                    g_arrive_tx(full_x(rx.s), x_bytes);    // K stages past the end are zero-filled
+                    g_tma_load_3d(x_tile(rx.s), &P.tmap_x, 0, m0, it.c * CS, full_x(rx.s));
+                } else {
+                    g_arrive_tx(full_x(rx.s), xs_bytes * (uint32_t)(it.hi - it.lo + 1));
+                    for (int k = it.lo; k <= it.hi; ++k)
+                        g_tma_load_2d(x_tile(rx.s) + (uint32_t)k * xs_bytes, &P.tmap_x, (it.c * CS + k) * kGemmBK, m0,
+                                      full_x(rx.s));
+                }
+            }
+            issued = it.seq + 1;
+        }
+        for (int64_t q = max((int64_t)0, issued - DX); q < issued; ++q)
+            if (!g_wait_warp(full_x((int)(q % DX)), (uint32_t)((q / DX) & 1))) ok = false;
+    } else if (warp == 1 || warp == 2) {
+        // -------------------------------------------------------- MMA --
+        const int j = warp - 1;
+        if (j < NI) {
+            const uint32_t acc = tmem + (uint32_t)j * P.acc_cols;
+            GRing rx, rw, rd;                              // X slot, W_hat slot, commit of the chunk
+            rx.init(DX);
+            rw.init(DW);
+            rd.init(DD);
+            uint32_t seg_ph = 0u;                          // parity of the epilogue's next acc_empty phase
+            bool fresh = true;                             // next MMA into acc starts a sum
+            int mine = 0;                                  // seq % NI, kept incrementally
+            for (; it.valid() && ok; it.next(), rx.next(), rw.next(), rd.next(), mine = mine + 1 == NI ? 0 : mine + 1) {
+                if (it.seg_first && it.seq > 0) {
+                    // a new segment: the epilogue must have read the previous one
+                    if (!g_wait_warp(acc_empty, seg_ph)) ok = false;
+                    seg_ph ^= 1u;
+                    fresh = true;
+                }
+                if (ok && mine == j) {
+                    if (!g_wait_warp(full_x(rx.s), rx.ph)) {
+                        ok = false;
+                        break;
+                    }
+                    for (int k = it.lo; k <= it.hi && ok; ++k) {
+                        if (!g_wait_warp(full_w(rw.s, k), rw.ph)) {
+                            ok = false;
+                            break;
+                        }
+                        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                        g_mma_stage_ts(acc, tmem + w_col0 + 32u * (uint32_t)(rw.s * CS + k),
+                                       x_tile(rx.s) + (uint32_t)k * xs_bytes, P.idesc, fresh ? 0u : 1u);
+                        fresh = false;
+                    }
+                    if (!ok) break;
+                    g_commit(done(rd.s));                  // frees the chunk's X slot and W_hat slot
+                }
+                if (ok && it.seg_last) g_commit(acc_full(j)); // the segment's sums (of this issuer) are complete
+            }
+            g_commit(fin + 8u * (uint32_t)j);
+            if (!g_wait_warp(fin + 8u * (uint32_t)j, 0u)) ok = false;
+        }
+    } else if (warp >= kGemmEpi0 && warp < kGemmEpi0 + 4) {
+        // --------------------------------------------------- epilogue --
+        const int quarter = warp & 3;
+        uint32_t par = 0u;
+        int64_t seg_seq0 = 0;
+        for (; it.valid() && ok; it.next()) {
+            if (it.seg_first) seg_seq0 = it.seq;
+            if (!it.seg_last) continue;
+            // issuers holding a partial sum of this segment
+            const int64_t len = it.seq - seg_seq0 + 1;
+            const int nacc = (int)min((int64_t)NI, len);
+            for (int a = 0; a < NI; ++a)
+                if (!g_wait_warp(acc_full(a), par)) ok = false;
+            par ^= 1u;
+            if (!ok) break;
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            const int64_t n = (it.tile / P.tiles_m) * kGemmBN + 32 * quarter + lane;
+            const int64_t m0 = (it.tile % P.tiles_m) * NT;
+            const int first_acc = (int)(seg_seq0 % NI);
+            const bool full = it.seg_full;
+            for (int c = 0; c < NT; c += 16) {
+                float v[16];
+                g_tmem_ld16(tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)first_acc * P.acc_cols + (uint32_t)c,
+                            v);
+                if (nacc == 2) {
+                    float v2[16];
+                    g_tmem_ld16(tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(1 - first_acc) * P.acc_cols +
+                                    (uint32_t)c,
+                                v2);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] = __fadd_rn(v[i], v2[i]);
+                }
+                if (n < P.N) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int64_t m = m0 + c + i;
+                        if (m < P.M) {
+                            float* dst = P.y + m * P.ldy + n;   // a warp writes 32 consecutive floats
+                            if (full) *dst = v[i];
+                            else atomicAdd(dst, v[i]);
+                        }
+                    }
+                }
+            }
+            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) g_arrive(acc_empty);
+        }
+    } else if (warp >= kGemmDq0) {
+        // ---------------------------------------------------- dequant --
+        const int grp = (warp - kGemmDq0) >> 2, quarter = warp & 3;
+        const int r = 32 * quarter + lane;                 // weight row of the tile, TMEM lane
+        const uint32_t lane_addr = tmem + ((uint32_t)(32 * quarter) << 16) + w_col0;
+        GRing rc, rw, rd;                                  // code slot, W_hat slot, commit of chunk seq - DW
+        rc.init(DC);
+        rw.init(DW);
+        rd.init(DD);
+        // group grp takes sub-stage grp % CS of the chunks with seq % (4 / CS) == grp / CS
+        const int cpg = kGemmGroups / CS, my_pc = grp / CS, k = grp % CS;
+        int pc = 0;                                        // seq % cpg, kept incrementally
+        int64_t cur_tile = -1;
+        GDeq deq{};
+        for (; it.valid() && ok; it.next(), rc.next(), rw.next(), pc = pc + 1 == cpg ? 0 : pc + 1) {
+            const bool reuse = it.seq >= DW;
+            const int rd_s = rd.s;
+            const uint32_t rd_ph = rd.ph;
+            if (reuse) rd.next();                          // now at chunk seq - DW + 1
+            if (pc != my_pc) continue;
+            // the W_hat slot is free once the commit of chunk seq - DW is in
+            if (reuse && !g_wait_warp(done(rd_s), rd_ph)) {
+                ok = false;
+                break;
+            }
+            if (k < it.lo || k > it.hi) {
+                // a sub-stage the block does not own: nothing to dequantize,
+                // but its W_hat barrier still completes a phase (keeping the
+                // slot's phases in step); the code slot's release for it was
+                // counted by the code producer
+                __syncwarp();
+                if (lane == 0) g_arrive(full_w(rw.s, k));
+                continue;
+            }
+            if (it.tile != cur_tile) {
+                cur_tile = it.tile;
+                const int64_t n = (it.tile / P.tiles_m) * kGemmBN + r;
+                const float srow = n < P.N ? __half2float(__ushort_as_half(P.scale[n])) : 0.0f;
+                deq = g_deq_consts(P.qbits, srow);
+            }
+            if (!g_wait_warp(full_c(rc.s), rc.ph)) {
                 ok = false;
                 break;
             }
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            // descriptors of the stage's K = 16 steps: 32 bytes apart within the swizzle atom
-            uint64_t da[4], db[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint64_t dx = g_smem_desc(x_tile(sx) + 32u * (uint32_t)i);
-                const uint64_t dw = g_smem_desc(w_tile(s) + 32u * (uint32_t)i);
-                da[i] = P.swap ? dw : dx;
-                db[i] = P.swap ? dx : dw;
-            }
-            g_mma_stage(acc, da, db, P.idesc, kt >= kGemmMmaWarps ? 1u : 0u);
-            g_commit(mma_done(kt));      // frees the stage's X and W_hat slots once these MMAs are done
-        }
-        g_commit(done);                  // also after a failure: lets the epilogue go
-    } else {
-        // ------------------------------------ W_hat tiles (dequant), epilogue --
-        // group gi takes stages gi, gi + 2, ...; two threads per weight row,
-        // the 8 lanes of a quarter warp on 8 consecutive rows with the same
-        // half (conflict-free swizzled stores)
-        const int t = threadIdx.x - 32 * kGemmDqWarp0;
-        const int gi = t / kGemmGroup, tg = t % kGemmGroup;
-        const int r = 8 * (tg >> 4) + (tg & 7), h = (tg >> 3) & 1;
-        const float srow = n0 + r < P.N ? __half2float(__ushort_as_half(P.scale[n0 + r])) : 0.0f;
-        const GDeq deq = g_deq_consts(P.qbits, srow);
-        const uint32_t code_off = row_code_bytes * (uint32_t)r + (row_code_bytes / 2u) * (uint32_t)h;
-        for (int kt = gi; kt < KT && ok; kt += kGemmDqGroups) {
-            const int s = kt % DW;
-            const int cs = kt % DC, g = kt / DC;
-            // the codes have landed; the slot's previous stage has been consumed
-            if (!g_wait(full_c(cs), (uint32_t)(g & 1)) ||
-                (kt >= DW && !g_wait(mma_done(kt - DW), done_parity(kt - DW)))) {
-                ok = false;
-                break;
-            }
-            const uint32_t dst = w_tile(s) + 128u * (uint32_t)r;
-            if (P.qbits == 6) g_dequant_part<6>(c_tile(cs) + code_off, empty_c(cs), dst, r, h, deq);
-            else g_dequant_part<8>(c_tile(cs) + code_off, empty_c(cs), dst, r, h, deq);
-            // generic-proxy writes -> visible to the tensor core (async proxy)
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            g_arrive(full_w(s));
-        }
-        if (!g_wait(done, 0u)) ok = false;
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        const int quarter = warp & 3;                      // TMEM lanes this warp may read
-        const int cpart = (warp - kGemmDqWarp0) >> 2;      // four warps per lane quarter
-        const int nacc = min(KT, kGemmMmaWarps);           // accumulators holding a partial sum
-        if (P.swap) {
-            // accumulator lane = weight row n, column = token m0 + j
-            const int64_t n = n0 + 32 * quarter + lane;
-            for (int c = cpart; c < P.nt / 16; c += 4) {
-                float v[16];
-                g_acc16(tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(16 * c), P.acc_cols, nacc, v);
-                if (n < P.N && ok) {
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int64_t m = m0 + 16 * c + j;
-                        if (m < P.M) {
-                            float* dst = P.y + m * P.ldy + n;   // a warp writes 32 consecutive floats
-                            if (P.accumulate) atomicAdd(dst, v[j]);
-                            else *dst = v[j];
-                        }
-                    }
-                }
-            }
-        } else {
-            // accumulator lane = token m, column = weight row n0 + j
-            const int64_t m = m0 + 32 * quarter + lane;
-            for (int c = cpart * (kGemmBN / 64); c < (cpart + 1) * (kGemmBN / 64); ++c) {
-                float v[16];
-                g_acc16(tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(16 * c), P.acc_cols, nacc, v);
-                if (m < P.M && ok) {
-                    float* yrow = P.y + m * P.ldy + n0 + 16 * c;
-#pragma unroll
-                    for (int j = 0; j < 16; j += 4) {
-                        const int64_t col = n0 + 16 * c + j;
-                        if (col + 3 < P.N) {
-                            if (P.accumulate) {
-                                asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(yrow + j),
-                                             "f"(v[j]), "f"(v[j + 1]),
-                                             "f"(v[j + 2]), "f"(v[j + 3])
-                                             : "memory");
-                            } else {
-                                *reinterpret_cast<float4*>(yrow + j) =
-                                    make_float4(v[j], v[j + 1],
-                                                v[j + 2], v[j + 3]);
-                            }
-                        } else {
-                            for (int e = 0; e < 4 && col + e < P.N; ++e) {   // the last columns of Y
-                                if (P.accumulate) atomicAdd(yrow + j + e, v[j + e]);
-                                else yrow[j + e] = v[j + e];
-                            }
-                        }
-                    }
-                }
+            const uint32_t codes = c_tile(rc.s) + (uint32_t)r * crow + (uint32_t)k * cb;
+            const uint32_t taddr = lane_addr + 32u * (uint32_t)(rw.s * CS + k);
+            if (P.qbits == 6) g_dequant_stage<6>(codes, taddr, deq);
+            else g_dequant_stage<8>(codes, taddr, deq);
+            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) {
+                g_arrive(empty_c(rc.s));                   // every lane's code loads have been used
+                g_arrive(full_w(rw.s, k));
             }
         }
     }
     if (!ok && lane == 0 && P.status) atomicOr(reinterpret_cast<unsigned int*>(P.status), 0x4u);
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
-    if (warp == 2) {
+    if (warp == 3) {
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(P.tmem_cols)
-                     : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
     }
 }
 

@@ -282,3 +282,16 @@ def unified11_gptq_inputs():
     four weights (unified projection, out-projection, MLP up, MLP down), in the
     order of unified11_train().specs."""
     return [s.shape[1] for s in unified11_train().specs]
+
+
+def random_packed_codes(rng, rows, row_bytes):
+    """Arbitrary packed code bytes [rows, row_bytes] (uint8): inputs for the
+    consuming GEMM, which accepts any 6- or 8-bit field."""
+    return rng.integers(0, 256, (rows, row_bytes), dtype=np.uint8)
+
+
+def random_f16_scales(rng, rows, lo=2.0 ** -12, hi=2.0 ** -5):
+    """Positive binary16 row scales as uint16 bit patterns, log-uniform in
+    [lo, hi] (normal binary16 numbers)."""
+    v = np.exp(rng.uniform(math.log(lo), math.log(hi), rows)).astype(np.float16)
+    return v.view(np.uint16)
