@@ -468,6 +468,20 @@ def measure_rows(gq, device, peak):
                2 * N * K + 2 * M * K + 2 * M * N, 2 * N * K, None,
                note="torch.matmul, bf16 W_hat read, bf16 Y; not counting the dequant pass", flops=fl)
         del q, X, Y, Wh
+    # the same GEMM with the fake-quant in the weight load (training forward),
+    # decode-sized batch over bf16 weights with training-mode row scales, and
+    # the 11-layer d528 model's two input widths
+    for M, N, K in ((16, 16384, 16384), (64, 1584, 528), (64, 528, 1584)):
+        Wb = synth.draw_bandwidth_matrix(N, K, 0, device=device).to(torch.bfloat16)
+        (cl,) = gq.row_clip_select([gq.Request(Wb, 6, 1.0)])
+        X = (torch.randn(M, K, device=device) * 0.5).to(torch.bfloat16)
+        Y = torch.empty(M, N, device=device)
+        wbytes = 2 * N * K + 4 * N
+        record(f"gemm fake-quant-on-load int6 from bf16 M{M} N{N} K{K}",
+               timed(lambda: gq.gemm_fakequant(X, Wb, cl.clip, 6, y=Y), flush_between=True),
+               wbytes + 2 * M * K + 4 * M * N, wbytes, 1,
+               note="bf16 weights + fp32 clips + bf16 X read, fp32 Y written", flops=2 * M * N * K)
+        del Wb, cl, X, Y
 
     # model-shaped batched workloads (L2-resident: flushed between reps)
     def oracle_time(items, export):
@@ -908,31 +922,43 @@ def run_reference(args, world, rank, local):
 
 
 def run_gemm(args):
-    """The dequant-on-load GEMM alone on one shape (``--gemm M,N,K,QBITS``):
-    synthetic weight exported through libgq, random bf16 X, ``warmup`` then
-    ``steps`` back-to-back calls timed with CUDA events.  An entry point for
-    profiling that kernel; it prints one JSON line of its own."""
+    """The consuming GEMM alone on one shape (``--gemm M,N,K,QBITS`` for the
+    dequant from packed codes, ``--gemm M,N,K,QBITS,bf16|f32`` for the
+    fake-quant from weights with training-mode scales): synthetic weight,
+    random bf16 X, ``warmup`` then ``steps`` back-to-back calls timed with
+    CUDA events.  An entry point for profiling; one JSON line of its own."""
     import torch
     from int6_int8_weight_b200 import gq
-    M, N, K, qbits = (int(v) for v in args.gemm.split(","))
+    parts = args.gemm.split(",")
+    M, N, K, qbits = (int(v) for v in parts[:4])
+    wmode = parts[4] if len(parts) > 4 else None
     device = torch.device("cuda")
     W = synth.draw_bandwidth_matrix(N, K, 0, device=device)
-    (q,) = gq.export_pack([gq.Request(W, qbits, 0.9999, want_dq=False)], check_status=False)
-    del W
     X = (torch.randn(M, K, device=device) * 0.5).to(torch.bfloat16)
     Y = torch.empty(M, N, device=device)
+    if wmode is None:
+        (q,) = gq.export_pack([gq.Request(W, qbits, 0.9999, want_dq=False)], check_status=False)
+        del W
+        fn = lambda: gq.gemm_dequant(X, q.packed, q.scale_f16, qbits, y=Y)  # noqa: E731
+        wbytes = q.packed.numel() + 2 * N
+        name = f"M{M} N{N} K{K} int{qbits}"
+    else:
+        Wm = W.to(torch.bfloat16) if wmode == "bf16" else W
+        (c,) = gq.row_clip_select([gq.Request(Wm, qbits, 1.0)])
+        fn = lambda: gq.gemm_fakequant(X, Wm, c.clip, qbits, y=Y)  # noqa: E731
+        wbytes = Wm.numel() * Wm.element_size() + 4 * N
+        name = f"M{M} N{N} K{K} fake-quant int{qbits} from {wmode}"
     for _ in range(args.warmup):
-        gq.gemm_dequant(X, q.packed, q.scale_f16, qbits, y=Y)
+        fn()
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
     for _ in range(args.steps):
-        gq.gemm_dequant(X, q.packed, q.scale_f16, qbits, y=Y)
+        fn()
     b.record()
     torch.cuda.synchronize()
     us = a.elapsed_time(b) * 1e3 / max(args.steps, 1)
-    wbytes = q.packed.numel() + 2 * N
-    print(json.dumps({"gemm": f"M{M} N{N} K{K} int{qbits}", "us_per_call": round(us, 2),
+    print(json.dumps({"gemm": name, "us_per_call": round(us, 2),
                       "tflops": round(2 * M * N * K / us / 1e6, 1),
                       "alg_gbs": round((wbytes + 2 * M * K + 4 * M * N) / us / 1e3, 1)}), flush=True)
 

@@ -297,20 +297,27 @@ GQ_API gq_status gq_dequant(const uint8_t* d_packed, const uint16_t* d_scale_f16
  * gq_packed_row_bytes(K, qbits) bytes, as gq_export_pack writes them for a
  * weight [N, K] exported per row) and s[n] = (float)scale_f16[n].  W_hat is
  * the bf16 fake-quant weight the forward pass would multiply by; it is
- * rebuilt tile by tile in shared memory and never written to memory.
+ * rebuilt tile by tile in tensor memory (the MMA's A operand) and never
+ * written out.
  *   d_x      bf16 [M, ldx] activations, row-major, 16-byte aligned, ldx % 8 == 0
- *   d_packed [N, gq_packed_row_bytes(K, qbits)] bytes, 16-byte aligned
+ *   d_packed [N, gq_packed_row_bytes(K, qbits)] bytes, 16-byte aligned (4-byte
+ *            aligned when the row length is not a multiple of 16 bytes)
  *   d_scale_f16 [N] binary16 bit patterns, 2-byte aligned
- *   d_y      fp32 [M, ldy] output, overwritten; 16-byte aligned, ldy % 4 == 0
+ *   d_y      fp32 [M, ldy] output, overwritten; 4-byte aligned, ldy >= N
  *   d_status nullable: set to 0 on the stream, then GQ_STATUS_TIMEOUT if a
  *            bounded wait on the device gave up (Y is then not valid)
  * All buffers are the caller's; the call allocates nothing, checks its
  * arguments on the host before launching, and runs asynchronously on
- * `stream` (one kernel launch, plus a memset of Y when K is split).
+ * `stream` (one kernel launch, plus a memset of Y when the batch has few
+ * tiles and their K ranges are split over blocks).
  * Products are exact (bf16 x bf16) and accumulate in binary32 in the tensor
- * cores' order, so Y is not bitwise reproducible against a sequential sum:
- * |Y - exact| <= (K/8 + 4) * 2^-24 * sum_k |X[m, k] * W_hat[n, k]|.
- * K must be a multiple of 64 (GQ_ERR_UNSUPPORTED otherwise).  Source: STE
+ * cores' order (two accumulators for small batches, partial sums of split K
+ * ranges added into Y), so Y is not bitwise reproducible against a sequential
+ * sum: |Y - exact| <= (K/8 + 16) * 2^-24 * sum_k |X[m, k] * W_hat[n, k]|.
+ * Any K: the last 64-wide stage is zero-filled.  Packed rows must be 4-byte
+ * aligned in length (int6: K % 16 == 0; int8: K % 4 == 0), else
+ * GQ_ERR_UNSUPPORTED; rows whose length is a multiple of 16 bytes arrive by
+ * TMA, others by 4-byte copies.  Source: STE
  * fake quantization in the forward pass whose weights feed the layer's
  * matmuls ("SubSixteen v2" page, Other; PR #1202, Quantization), with the
  * int6 / int8 storage of the export (PR #1495, Mixed-bit quantization).
@@ -384,6 +391,30 @@ GQ_API gq_status gq_gptq_quantize(const gq_tensor* t, const double* d_H, double 
  */
 GQ_API gq_status gq_gptq_hessian(const void* d_x, int32_t dtype, int64_t n, int64_t cols, int64_t ldx,
                                  double* d_H, int accumulate, cudaStream_t stream);
+
+/*
+ * The consuming GEMM of quantization-aware training, with the fake-quant in
+ * its weight load:
+ *   Y[m, n] = sum_k X[m, k] * W_hat[n, k],  W_hat[n, k] = bf16(RN(q[n, k] * s[n])),
+ *   q = clamp(round_half_even(clip(w[n, k], -c[n], c[n]) / s[n]), -qmax, qmax),
+ *   s[n] = c[n] / qmax (GQ_SCALE_F32) or binary16(c[n] / qmax) (GQ_SCALE_F16),
+ * i.e. exactly the w_hat that gq_fakequant_fwd writes for the same weight and
+ * clips (for fp32 weights, that w_hat rounded once to bf16 for the tensor
+ * cores), rebuilt tile by tile in tensor memory and never written out.
+ *   d_x      bf16 [M, ldx], 16-byte aligned, ldx % 8 == 0
+ *   d_w      w_dtype (GQ_F32 / GQ_BF16) [N, ldw] row-major, 16-byte aligned,
+ *            ldw * element size a multiple of 16
+ *   d_clip   binary32 [N] row clips c, e.g. from gq_row_clip_select
+ *   d_y, ldy, d_status, accumulation and error bound as gq_gemm_dequant;
+ *   any K.  d_status also receives GQ_STATUS_RANGE for a binary16 scale
+ *   overflow (GQ_SCALE_F16).
+ * Source: STE fake quantization in the forward pass ("SubSixteen v2", Other;
+ * PR #1202, Quantization: STE QAT, bits 6, scope all).
+ */
+GQ_API gq_status gq_gemm_fakequant(const void* d_x, int64_t M, int64_t K, int64_t ldx, const void* d_w,
+                                   int32_t w_dtype, int64_t ldw, const float* d_clip, int qbits,
+                                   gq_scale_mode mode, int64_t N, float* d_y, int64_t ldy, int32_t* d_status,
+                                   cudaStream_t stream);
 
 /* Device workspace bytes a batch needs (0 when it has no per-tensor group). */
 GQ_API size_t gq_workspace_size(const gq_tensor* t, int n);

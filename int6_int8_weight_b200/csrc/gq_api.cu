@@ -509,7 +509,7 @@ gq_status quantize_batch(const gq_tensor* t, int n, Op op, bool f16_mode, void* 
 // ---------------------------------------------------- dequant-on-load GEMM --
 
 std::atomic<void*> g_encode_tiled{nullptr};
-std::atomic<int> g_gemm_smem_set[kMaxDevices];
+std::atomic<int> g_gemm_smem_set[2][kMaxDevices];
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no
 // link-time dependency on the driver library).
@@ -584,6 +584,171 @@ GptqWs gptq_layout(void* base, int64_t rows, int64_t cols) {
 }
 
 std::atomic<int> g_gptq_smem_set[kMaxDevices];
+
+struct GemmIn {
+    const void* x;
+    int64_t M, K, ldx, N, ldy;
+    float* y;
+    int32_t* status;
+    cudaStream_t stream;
+    int qbits, wmode;                 // wmode 0: packed codes; 1 / 2: bf16 / fp32 weights + clip
+    const uint8_t* packed;
+    const uint16_t* scale;
+    int64_t prb;
+    bool tma_codes;
+    const void* w;
+    int64_t ldw;
+    const float* clip;
+    int export_scale;
+};
+
+// The launch shared by the dequant-on-load and the fake-quant-on-load GEMM
+// (arguments already checked).
+gq_status gemm_launch(const GemmIn& in) {
+    const void* d_x = in.x;
+    const int64_t M = in.M, K = in.K, ldx = in.ldx, N = in.N, ldy = in.ldy;
+    float* d_y = in.y;
+    int32_t* d_status = in.status;
+    cudaStream_t stream = in.stream;
+    const int qbits = in.qbits;
+    const uint8_t* d_packed = in.packed;
+    const uint16_t* d_scale_f16 = in.scale;
+    const int64_t prb = in.prb;
+    const bool tma_codes = in.tma_codes;
+    PFN_cuTensorMapEncodeTiled enc = encode_tiled();
+    if (!enc) return GQ_ERR_UNSUPPORTED;
+    GemmParams P;
+    std::memset(&P, 0, sizeof(P));
+    // token tile: the batch itself up to 256 tokens (rounded up to 16 .. 256), else 256
+    int nt = 16;
+    while (nt < M && nt < 256) nt *= 2;
+    P.nt = nt;
+    P.ni = nt <= 64 ? 2 : 1;
+    // K stages per code copy / W_hat chunk / MMA commit, and per X copy (at
+    // most 32 KB); the weight modes copy one stage of weights at a time
+    P.cs = in.wmode ? 1 : 4;
+    P.xs = in.wmode ? 1 : nt <= 64 ? 4 : nt == 128 ? 2 : 1;
+    P.wmode = in.wmode;
+    P.idesc = gemm_idesc(kGemmBN, (uint32_t)nt);
+    P.acc_cols = (uint32_t)std::max(32, nt);
+    const cuuint32_t estride[3] = {1, 1, 1};
+    // X: a 3-D view {64, M, K / 64} (one copy per chunk) when K % 64 == 0,
+    // else the 2-D [M, K] view (one copy per stage)
+    P.x3d = 0;
+    if (K % kGemmBK == 0) {
+        const cuuint64_t gdim3[3] = {(cuuint64_t)kGemmBK, (cuuint64_t)M, (cuuint64_t)(K / kGemmBK)};
+        const cuuint64_t gstride3[2] = {(cuuint64_t)ldx * 2, (cuuint64_t)kGemmBK * 2};
+        const cuuint32_t box3[3] = {(cuuint32_t)kGemmBK, (cuuint32_t)nt, (cuuint32_t)P.xs};
+        if (enc(&P.tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(d_x), gdim3, gstride3, box3, estride,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+            P.x3d = 1;
+    }
+    if (!P.x3d) {
+        const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)M};
+        const cuuint64_t gstride[1] = {(cuuint64_t)ldx * 2};
+        const cuuint32_t box[2] = {(cuuint32_t)kGemmBK, (cuuint32_t)nt};
+        if (enc(&P.tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(d_x), gdim, gstride, box, estride,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return GQ_ERR_UNSUPPORTED;
+    }
+    // bytes of a row's 64-wide stage in a code slot (codes, or bf16 / fp32 weights)
+    const int64_t cb = in.wmode == 1 ? 128 : in.wmode == 2 ? 256 : qbits == 6 ? 48 : 64;
+    const int64_t crow = cb * P.cs;                   // ... of a row's chunk
+    if (in.wmode == 1) {
+        // bf16 weights [N, ldw]: box 64 x 128 (128-byte rows), 128-byte swizzle
+        const cuuint64_t wdim[2] = {(cuuint64_t)K, (cuuint64_t)N};
+        const cuuint64_t wstride[1] = {(cuuint64_t)in.ldw * 2};
+        const cuuint32_t wbox[2] = {(cuuint32_t)kGemmBK, (cuuint32_t)kGemmBN};
+        if (enc(&P.tmap_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(in.w), wdim, wstride, wbox, estride,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return GQ_ERR_UNSUPPORTED;
+    } else if (in.wmode == 2) {
+        // fp32 weights: a stage is two 32-wide halves (128-byte rows); one
+        // 3-D copy {32, 128, 2} of the view {32, N, K / 32} when K % 32 == 0,
+        // else two 2-D copies (the tail zero-filled)
+        P.w3d = 0;
+        if (K % 32 == 0) {
+            const cuuint64_t wdim3[3] = {32, (cuuint64_t)N, (cuuint64_t)(K / 32)};
+            const cuuint64_t wstride3[2] = {(cuuint64_t)in.ldw * 4, 128};
+            const cuuint32_t wbox3[3] = {32, (cuuint32_t)kGemmBN, 2};
+            if (enc(&P.tmap_w, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(in.w), wdim3, wstride3, wbox3,
+                    estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+                P.w3d = 1;
+        }
+        if (!P.w3d) {
+            const cuuint64_t wdim[2] = {(cuuint64_t)K, (cuuint64_t)N};
+            const cuuint64_t wstride[1] = {(cuuint64_t)in.ldw * 4};
+            const cuuint32_t wbox[2] = {32, (cuuint32_t)kGemmBN};
+            if (enc(&P.tmap_w, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(in.w), wdim, wstride, wbox,
+                    estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                return GQ_ERR_UNSUPPORTED;
+        }
+    } else if (tma_codes) {
+        const cuuint64_t wdim[2] = {(cuuint64_t)prb, (cuuint64_t)N};
+        const cuuint64_t wstride[1] = {(cuuint64_t)prb};
+        const cuuint32_t wbox[2] = {(cuuint32_t)crow, (cuuint32_t)kGemmBN};
+        if (enc(&P.tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(d_packed), wdim, wstride, wbox,
+                estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return GQ_ERR_UNSUPPORTED;
+    }
+    P.code_copy = (in.wmode == 0 && !tma_codes) ? 1 : 0;
+    P.codes = d_packed;
+    P.scale = d_scale_f16;
+    P.clip = in.clip;
+    P.export_scale = in.export_scale;
+    P.y = d_y;
+    P.status = d_status;
+    P.M = M;
+    P.N = N;
+    P.K = K;
+    P.ldy = ldy;
+    P.prb = prb;
+    P.qbits = qbits;
+    P.kt_per_tile = (int32_t)((K + kGemmBK - 1) / kGemmBK);
+    const int64_t tiles_n = (N + kGemmBN - 1) / kGemmBN, tiles_m = (M + nt - 1) / nt;
+    P.tiles_m = (int32_t)tiles_m;
+    P.tiles = tiles_n * tiles_m;
+    const int64_t sms = sm_count();
+    // few tiles: split the stage units evenly (partial sums added into a
+    // zeroed Y); many: whole tiles round-robin
+    P.streamk = P.tiles < 2 * sms ? 1 : 0;
+    const int64_t units = P.streamk ? P.tiles * P.kt_per_tile : P.tiles;
+    const int64_t grid = std::min<int64_t>(sms, units);
+    // ring depths in chunks: X up to 64 KB (at least 2 slots), codes in what
+    // is left, W_hat in the TMEM columns after the accumulators; the commit
+    // ring is a multiple of the W_hat depth and at least the X depth (a
+    // waiter on any of these barriers then never sees a phase two ahead)
+    const int64_t x_bytes = (int64_t)nt * 128 * P.xs, c_bytes = kGemmBN * crow;
+    // codes: 3 chunks (12 stages) for wide token tiles, else up to 6; X slots
+    // in the rest (at most 8)
+    const int64_t dc_want = in.wmode ? (in.wmode == 1 ? 6 : 4) : nt >= 128 ? 3 : 6;
+    P.dc = (int32_t)std::min<int64_t>(dc_want, (kGemmRingBytes - 2 * x_bytes) / c_bytes);
+    P.dx = (int32_t)std::min<int64_t>(in.wmode ? 12 : 8, (kGemmRingBytes - P.dc * c_bytes) / x_bytes);
+    P.dw = (int32_t)std::min<int64_t>(kGemmMaxWS / P.cs, (512 - P.ni * (int64_t)P.acc_cols) / (32 * P.cs));
+    P.dd = P.dw;                                        // the commit ring frees W_hat slots only
+    if (P.dc < 2 || P.dw < 2 || P.dx < 2 || P.dd > kGemmMaxDone || P.dx > kGemmMaxX) return GQ_ERR_UNSUPPORTED;
+    if (P.streamk &&
+        cuda_status(cudaMemset2DAsync(d_y, (size_t)ldy * 4, 0, (size_t)N * 4, (size_t)M, stream)) != GQ_OK)
+        return GQ_ERR_CUDA;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GQ_ERR_CUDA;
+    const int wi = in.wmode ? 1 : 0;
+    if (dev >= 0 && dev < kMaxDevices && g_gemm_smem_set[wi][dev].load() < kGemmSmemBytes) {
+        if (cuda_status(cudaFuncSetAttribute(wi ? gemm_dequant_kernel<1> : gemm_dequant_kernel<0>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes)) != GQ_OK)
+            return GQ_ERR_CUDA;
+        g_gemm_smem_set[wi][dev].store(kGemmSmemBytes);
+    }
+    if (wi) gemm_dequant_kernel<1><<<(unsigned)grid, kGemmThreads, kGemmSmemBytes, stream>>>(P);
+    else gemm_dequant_kernel<0><<<(unsigned)grid, kGemmThreads, kGemmSmemBytes, stream>>>(P);
+    return launch_status();
+}
 
 }  // namespace
 
@@ -799,95 +964,36 @@ gq_status gq_gemm_dequant(const void* d_x, int64_t M, int64_t K, int64_t ldx, co
         return GQ_ERR_MISALIGNED;
     if (K == 0)
         return cuda_status(cudaMemset2DAsync(d_y, (size_t)ldy * 4, 0, (size_t)N * 4, (size_t)M, stream));
-    PFN_cuTensorMapEncodeTiled enc = encode_tiled();
-    if (!enc) return GQ_ERR_UNSUPPORTED;
-    GemmParams P;
-    std::memset(&P, 0, sizeof(P));
-    // token tile: the batch itself up to 256 tokens (rounded up to 16 .. 256), else 256
-    int nt = 16;
-    while (nt < M && nt < 256) nt *= 2;
-    P.nt = nt;
-    P.ni = nt <= 64 ? 2 : 1;
-    P.cs = nt <= 128 ? 4 : 2;                           // K stages per copy (an X chunk of at most 64 KB)
-    P.idesc = gemm_idesc(kGemmBN, (uint32_t)nt);
-    P.acc_cols = (uint32_t)std::max(32, nt);
-    const cuuint32_t estride[3] = {1, 1, 1};
-    // X: a 3-D view {64, M, K / 64} (one copy per chunk) when K % 64 == 0,
-    // else the 2-D [M, K] view (one copy per stage)
-    P.x3d = 0;
-    if (K % kGemmBK == 0) {
-        const cuuint64_t gdim3[3] = {(cuuint64_t)kGemmBK, (cuuint64_t)M, (cuuint64_t)(K / kGemmBK)};
-        const cuuint64_t gstride3[2] = {(cuuint64_t)ldx * 2, (cuuint64_t)kGemmBK * 2};
-        const cuuint32_t box3[3] = {(cuuint32_t)kGemmBK, (cuuint32_t)nt, (cuuint32_t)P.cs};
-        if (enc(&P.tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(d_x), gdim3, gstride3, box3, estride,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
-            P.x3d = 1;
-    }
-    if (!P.x3d) {
-        const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)M};
-        const cuuint64_t gstride[1] = {(cuuint64_t)ldx * 2};
-        const cuuint32_t box[2] = {(cuuint32_t)kGemmBK, (cuuint32_t)nt};
-        if (enc(&P.tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(d_x), gdim, gstride, box, estride,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return GQ_ERR_UNSUPPORTED;
-    }
-    const int64_t cb = qbits == 6 ? 48 : 64;          // code bytes of a row's 64-code stage
-    const int64_t crow = cb * P.cs;                   // ... of a row's chunk
-    if (tma_codes) {
-        const cuuint64_t wdim[2] = {(cuuint64_t)prb, (cuuint64_t)N};
-        const cuuint64_t wstride[1] = {(cuuint64_t)prb};
-        const cuuint32_t wbox[2] = {(cuuint32_t)crow, (cuuint32_t)kGemmBN};
-        if (enc(&P.tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(d_packed), wdim, wstride, wbox,
-                estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return GQ_ERR_UNSUPPORTED;
-    }
-    P.code_copy = tma_codes ? 0 : 1;
-    P.codes = d_packed;
-    P.scale = d_scale_f16;
-    P.y = d_y;
-    P.status = d_status;
-    P.M = M;
-    P.N = N;
-    P.K = K;
-    P.ldy = ldy;
-    P.prb = prb;
-    P.qbits = qbits;
-    P.kt_per_tile = (int32_t)((K + kGemmBK - 1) / kGemmBK);
-    const int64_t tiles_n = (N + kGemmBN - 1) / kGemmBN, tiles_m = (M + nt - 1) / nt;
-    P.tiles_m = (int32_t)tiles_m;
-    P.tiles = tiles_n * tiles_m;
-    const int64_t sms = sm_count();
-    // few tiles: split the stage units evenly (partial sums added into a
-    // zeroed Y); many: whole tiles round-robin
-    P.streamk = P.tiles < 2 * sms ? 1 : 0;
-    const int64_t units = P.streamk ? P.tiles * P.kt_per_tile : P.tiles;
-    const int64_t grid = std::min<int64_t>(sms, units);
-    // ring depths in chunks: X up to 64 KB (at least 2 slots), codes in what
-    // is left, W_hat in the TMEM columns after the accumulators; the commit
-    // ring is a multiple of the W_hat depth and at least the X depth (a
-    // waiter on any of these barriers then never sees a phase two ahead)
-    const int64_t x_bytes = (int64_t)nt * 128 * P.cs, c_bytes = kGemmBN * crow;
-    P.dx = (int32_t)std::max<int64_t>(2, std::min<int64_t>(8, (64 * 1024) / x_bytes));
-    P.dc = (int32_t)std::min<int64_t>(kGemmMaxC, (kGemmRingBytes - P.dx * x_bytes) / c_bytes);
-    P.dw = (int32_t)std::min<int64_t>(kGemmMaxW, (512 - P.ni * (int64_t)P.acc_cols) / (32 * P.cs));
-    P.dd = P.dw * ((P.dx + P.dw - 1) / P.dw);
-    if (P.dc < 2 || P.dw < 2 || P.dd > kGemmMaxDone || P.dx > kGemmMaxX) return GQ_ERR_UNSUPPORTED;
-    if (P.streamk &&
-        cuda_status(cudaMemset2DAsync(d_y, (size_t)ldy * 4, 0, (size_t)N * 4, (size_t)M, stream)) != GQ_OK)
-        return GQ_ERR_CUDA;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return GQ_ERR_CUDA;
-    if (dev >= 0 && dev < kMaxDevices && g_gemm_smem_set[dev].load() < kGemmSmemBytes) {
-        if (cuda_status(cudaFuncSetAttribute(gemm_dequant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kGemmSmemBytes)) != GQ_OK)
-            return GQ_ERR_CUDA;
-        g_gemm_smem_set[dev].store(kGemmSmemBytes);
-    }
-    gemm_dequant_kernel<<<(unsigned)grid, kGemmThreads, kGemmSmemBytes, stream>>>(P);
-    return launch_status();
+    GemmIn in{};
+    in.x = d_x; in.M = M; in.K = K; in.ldx = ldx; in.N = N; in.y = d_y; in.ldy = ldy; in.status = d_status;
+    in.stream = stream; in.qbits = qbits; in.wmode = 0; in.packed = d_packed; in.scale = d_scale_f16;
+    in.prb = prb; in.tma_codes = tma_codes;
+    return gemm_launch(in);
+}
+
+gq_status gq_gemm_fakequant(const void* d_x, int64_t M, int64_t K, int64_t ldx, const void* d_w, int32_t w_dtype,
+                            int64_t ldw, const float* d_clip, int qbits, gq_scale_mode mode, int64_t N, float* d_y,
+                            int64_t ldy, int32_t* d_status, cudaStream_t stream) {
+    if (M < 0 || N < 0 || K < 0 || (qbits != 6 && qbits != 8)) return GQ_ERR_INVALID_ARG;
+    if (w_dtype != GQ_F32 && w_dtype != GQ_BF16) return GQ_ERR_INVALID_ARG;
+    if (mode != GQ_SCALE_F32 && mode != GQ_SCALE_F16) return GQ_ERR_INVALID_ARG;
+    if (ldx < K || ldw < K || ldy < N) return GQ_ERR_INVALID_ARG;
+    if (M > INT32_MAX || K > INT32_MAX || N > INT32_MAX) return GQ_ERR_UNSUPPORTED;
+    if (d_status && !aligned(d_status, 4)) return GQ_ERR_MISALIGNED;
+    if (d_status && cuda_status(cudaMemsetAsync(d_status, 0, sizeof(int32_t), stream)) != GQ_OK) return GQ_ERR_CUDA;
+    if (M == 0 || N == 0) return GQ_OK;
+    if (!d_x || !d_w || !d_clip || !d_y) return GQ_ERR_INVALID_ARG;
+    const int64_t esz = w_dtype == GQ_F32 ? 4 : 2;
+    if (!aligned(d_x, 16) || (ldx % 8) != 0 || !aligned(d_w, 16) || ((ldw * esz) % 16) != 0 || !aligned(d_clip, 4) ||
+        !aligned(d_y, 4))
+        return GQ_ERR_MISALIGNED;
+    if (K == 0)
+        return cuda_status(cudaMemset2DAsync(d_y, (size_t)ldy * 4, 0, (size_t)N * 4, (size_t)M, stream));
+    GemmIn in{};
+    in.x = d_x; in.M = M; in.K = K; in.ldx = ldx; in.N = N; in.y = d_y; in.ldy = ldy; in.status = d_status;
+    in.stream = stream; in.qbits = qbits; in.wmode = w_dtype == GQ_BF16 ? 1 : 2; in.w = d_w; in.ldw = ldw;
+    in.clip = d_clip; in.export_scale = mode == GQ_SCALE_F16 ? 1 : 0;
+    return gemm_launch(in);
 }
 
 size_t gq_workspace_size(const gq_tensor* t, int n) {

@@ -29,10 +29,12 @@
 //
 // Chunks.  One thread can start a TMA copy only about every 250 ns, whatever
 // its size, so copies move CS consecutive K stages at once (a chunk: CS = 4
-// for token tiles of up to 128, 2 for 256): one copy of the code rows
-// (128 rows x CS * 48 / 64 bytes) and one copy of the token tile (a 3-D
-// view of X, {64, nt, CS} with the 128-byte swizzle, when K % 64 == 0; else
-// one 2-D copy per stage).  A chunk is also the unit of the MMA hand-off:
+// for packed codes; 1 for the fake-quant modes, whose stage of bf16 / fp32
+// weights is already 16 / 32 KB): one copy of the code rows (128 rows x
+// CS * 48 / 64 bytes) and, per X slot of XS stages (XS = 4, 2, 1 for token
+// tiles of <= 64, 128, 256), one copy of the token tile (a 3-D view of X,
+// {64, nt, XS} with the 128-byte swizzle, when K % 64 == 0; else one 2-D
+// copy per stage).  A chunk is also the unit of the MMA hand-off:
 // one issuer runs all of a chunk's stages and commits once.  Chunks are
 // aligned to the tile's K stages; a block's first and last chunk of a tile
 // may hold only part of their stages (the copies still move the whole chunk).
@@ -65,9 +67,9 @@ constexpr int kGemmEpi0 = 4;                             // first epilogue warp
 constexpr int kGemmThreads = 32 * (kGemmDq0 + 4 * kGemmGroups);
 constexpr int kGemmMaxX = 16;                            // X chunk slots (max)
 constexpr int kGemmMaxC = 16;                            // code chunk slots (max)
-constexpr int kGemmMaxW = 4;                             // W_hat chunk slots in TMEM (max)
+constexpr int kGemmMaxWS = 16;                           // W_hat stage slots in TMEM (chunk slots x stages, max)
 constexpr int kGemmMaxDone = 32;                         // per-chunk MMA commit ring (max)
-constexpr int kGemmBarBytes = 8 * (kGemmMaxX + 2 * kGemmMaxC + kGemmMaxW * kGemmCSMax + kGemmMaxDone + 8) + 64;
+constexpr int kGemmBarBytes = 8 * (2 * kGemmMaxX + 2 * kGemmMaxC + kGemmMaxWS + kGemmMaxDone + 8) + 64;
 constexpr int kGemmSmemBytes = 232448;                   // all of it: 227 KB
 constexpr int kGemmRingBytes = kGemmSmemBytes - 1024 /* alignment */ - kGemmBarBytes;
 constexpr unsigned long long kGemmWaitNs = 4000000000ull;
@@ -76,14 +78,19 @@ struct GemmParams {
     CUtensorMap tmap_x;          // X: 3-D {64, M, K / 64} box {64, nt, CS}, or 2-D [M, K] box {64, nt}; SWIZZLE_128B
     CUtensorMap tmap_w;          // codes [N, prb] bytes, box (CS stages' bytes) x 128, no swizzle (TMA mode)
     const uint8_t* codes;        // packed codes (copy mode)
-    const uint16_t* scale;       // [N] binary16 row scales
+    const uint16_t* scale;       // [N] binary16 row scales (codes)
+    const float* clip;           // [N] row clips (weight modes)
+    int32_t wmode;               // 0: packed codes; 1: bf16 weights; 2: fp32 weights (fake-quant on load)
+    int32_t w3d;                 // fp32 weights: 1 = one 3-D copy {32, 128, 2} per stage, 0 = two 2-D copies
+    int32_t export_scale;        // weight modes: 1 = binary16 row scales, 0 = binary32
     float* y;                    // [M, ldy] fp32
     int32_t* status;             // nullable: GQ_STATUS_TIMEOUT on an expired wait
     int64_t M, N, K, ldy, prb;
     int32_t qbits;
     int32_t code_copy;           // 1: codes by cp.async (prb % 16 != 0), 0: by TMA
-    int32_t x3d;                 // 1: one 3-D copy of X per chunk, 0: one 2-D copy per stage
-    int32_t cs;                  // stages per chunk
+    int32_t x3d;                 // 1: one 3-D copy of X per X slot, 0: one 2-D copy per stage
+    int32_t cs;                  // stages per chunk (codes, W_hat, MMA commits)
+    int32_t xs;                  // stages per X slot (divides cs)
     int32_t kt_per_tile;         // 64-wide K stages per tile
     int32_t tiles_m;             // token tiles
     int64_t tiles;               // tiles_n * tiles_m
@@ -92,7 +99,7 @@ struct GemmParams {
     int32_t ni;                  // MMA issuers (accumulators)
     uint32_t idesc;              // tcgen05 instruction descriptor
     uint32_t acc_cols;           // TMEM columns of one accumulator
-    int32_t dx, dc, dw, dd;      // ring depths in chunks: X, codes, W_hat (TMEM), MMA commits
+    int32_t dx, dc, dw, dd;      // ring depths: X slots; chunks of codes, W_hat (TMEM), MMA commits
 };
 
 // ------------------------------------------------------------- PTX glue --
@@ -107,14 +114,18 @@ __device__ __forceinline__ unsigned long long g_now() {
     return t;
 }
 
+// Test for the completion of the phase with the given parity; a thread that
+// finds it incomplete may be suspended in the barrier for up to the hint
+// (20 us) until it completes, so that waiting warps leave the issue slots to
+// the working ones (24 warps share four schedulers).
 __device__ __forceinline__ bool g_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t done;
     asm volatile(
         "{\n .reg .pred p;\n"
-        " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
         " selp.u32 %0, 1, 0, p;\n}"
         : "=r"(done)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "r"(20000u)
         : "memory");
     return done != 0;
 }
@@ -125,7 +136,7 @@ __device__ __forceinline__ bool g_wait(uint32_t bar, uint32_t parity) {
     const unsigned long long t0 = g_now();
     for (uint32_t i = 1;; ++i) {
         if (g_try_wait(bar, parity)) return true;
-        if ((i & 63u) == 0u && g_now() - t0 > kGemmWaitNs) return false;
+        if ((i & 3u) == 0u && g_now() - t0 > kGemmWaitNs) return false;
     }
 }
 
@@ -200,6 +211,9 @@ __host__ __device__ constexpr uint32_t gemm_idesc(uint32_t m, uint32_t n) {
 // swizzle atom), issued by one elected lane from a single asm block.
 __device__ __forceinline__ void g_mma_stage_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_addr, uint32_t idesc,
                                                uint32_t accumulate) {
+    // 32 bytes further inside the swizzle atom is +2 in the descriptor's
+    // address field (addresses stay below 256 KB: no carry out of it)
+    const uint64_t b0 = g_smem_desc(b_addr);
     asm volatile(
         "{\n\t.reg .pred p, e;\n\t"
         "setp.ne.b32 p, %9, 0;\n\t"
@@ -209,8 +223,8 @@ __device__ __forceinline__ void g_mma_stage_ts(uint32_t d_tmem, uint32_t a_tmem,
         "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %7, %10, 1;\n\t"
         "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %8, %10, 1;\n\t"
         "}\n" ::"r"(d_tmem),
-        "r"(a_tmem), "r"(a_tmem + 8u), "r"(a_tmem + 16u), "r"(a_tmem + 24u), "l"(g_smem_desc(b_addr)),
-        "l"(g_smem_desc(b_addr + 32u)), "l"(g_smem_desc(b_addr + 64u)), "l"(g_smem_desc(b_addr + 96u)),
+        "r"(a_tmem), "r"(a_tmem + 8u), "r"(a_tmem + 16u), "r"(a_tmem + 24u), "l"(b0), "l"(b0 + 2u), "l"(b0 + 4u),
+        "l"(b0 + 6u),
         "r"(accumulate), "r"(idesc)
         : "memory");
 }
@@ -269,10 +283,10 @@ __device__ __forceinline__ uint64_t g_f2(float lo, float hi) {
 // significant bits, S_p is s scaled by a power of two, and C_p * S_p is
 // exact because C_p has at most 13 significant bits (p >= 6 for int6,
 // p >= 4 for int8) against the 11 of a binary16 s.  The only rounding is
-// the final one to bf16.  int6 takes fields at p = 12 and p = 6 (two codes
-// per 12-bit view of the code stream), int8 at p = 8, 4 and 12.
+// the final one to bf16.  int6 takes the two codes of a pair at p = 6 and
+// p = 12 of one view of the code stream, int8 at p = 8, 4 and 12.
 struct GDeq {
-    uint64_t s_a, c_a;           // int6 (S12, S6) / int8 even pair (S8, S8), and -C_p * S_p
+    uint64_t s_a, c_a;           // int6 (S6, S12) / int8 even pair (S8, S8), and -C_p * S_p
     uint64_t s_b, c_b;           // int8 odd pair (S4, S12)
 };
 
@@ -283,8 +297,8 @@ __device__ __forceinline__ GDeq g_deq_consts(int qbits, float s) {
     };
     GDeq d;
     if (qbits == 6) {
-        d.s_a = g_f2(sp(12), sp(6));
-        d.c_a = g_f2(cs(6, 12), cs(6, 6));
+        d.s_a = g_f2(sp(6), sp(12));
+        d.c_a = g_f2(cs(6, 6), cs(6, 12));
         d.s_b = d.c_b = 0;
     } else {
         d.s_a = g_f2(sp(8), sp(8));
@@ -314,18 +328,16 @@ __device__ __forceinline__ uint32_t g_pair_bf16(float f0, float f1, uint64_t s2,
 template <int QBITS>
 __device__ __forceinline__ uint32_t g_pair(const uint32_t (&w)[16], int i, const GDeq& d) {
     if constexpr (QBITS == 6) {
-        // the code stream shifted right by 12 (i - 1) holds code 2i at bit
-        // 12; shifted by 12 i it holds code 2i + 1 at bit 6
-        const int sh = 12 * i;
-        const uint32_t vb = __funnelshift_r(w[sh >> 5], w[(sh >> 5) + 1], sh & 31);
-        uint32_t va;
+        // the code stream shifted right by 12 i - 6 holds code 2i at bit 6
+        // and code 2i + 1 at bit 12: one funnel shift per pair
+        uint32_t v;
         if (i == 0) {
-            va = w[0] << 12;
+            v = w[0] << 6;
         } else {
-            const int sa = sh - 12;
-            va = __funnelshift_r(w[sa >> 5], w[(sa >> 5) + 1], sa & 31);
+            const int sh = 12 * i - 6;
+            v = __funnelshift_r(w[sh >> 5], w[(sh >> 5) + 1], sh & 31);
         }
-        return g_pair_bf16(g_field(va, 0x3F000u, 0x4B020000u), g_field(vb, 0xFC0u, 0x4B000800u), d.s_a, d.c_a);
+        return g_pair_bf16(g_field(v, 0xFC0u, 0x4B000800u), g_field(v, 0x3F000u, 0x4B020000u), d.s_a, d.c_a);
     } else {
         const uint32_t wd = w[i >> 1];
         if ((i & 1) == 0)                                  // bytes 0, 1: both at bit 8
@@ -362,6 +374,42 @@ __device__ __forceinline__ void g_dequant_stage(uint32_t codes, uint32_t taddr, 
         uint32_t out[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) out[j] = g_pair<QBITS>(w, 16 * h + j, d);
+        g_tmem_st16(taddr + 16u * (uint32_t)h, out);
+    }
+}
+
+// One weight row's 64-wide stage, fake-quantized on the way into TMEM:
+// w_hat = RN(q * s) with q = clamp(round_half_even(clip(w, -c, c) / s)), the
+// very arithmetic of the fused row kernel (quantize_offset / offset_to_dq),
+// then rounded to bf16 for the tensor cores.  The stage sits in shared
+// memory as 128-byte rows with the 128-byte swizzle (16-byte chunk j of row r
+// at chunk position j ^ (r & 7)): one row of 64 bf16, or two rows of 32 fp32
+// in halves 16 KB apart.
+template <int DT>
+__device__ __forceinline__ void g_fakequant_stage(uint32_t tile, int r, uint32_t taddr, const Scale& S) {
+    const uint32_t sw = (uint32_t)(r & 7), row = tile + 128u * (uint32_t)r;
+    auto fq = [&](float w) { return offset_to_dq(quantize_offset(w, S), S); };
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {                          // 32 weights -> 16 bf16x2 columns
+        uint32_t out[16];
+#pragma unroll
+        for (int c = 0; c < (DT == kBF16 ? 4 : 8); ++c) {
+            uint32_t u[4];
+            const uint32_t j = DT == kBF16 ? (uint32_t)(4 * h + c) : (uint32_t)c;
+            const uint32_t src = (DT == kBF16 ? row : row + (uint32_t)h * 128u * kGemmBN) + ((j ^ sw) << 4);
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3])
+                         : "r"(src)
+                         : "memory");
+            if constexpr (DT == kBF16) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    out[4 * c + e] = g_bf16x2(fq(__uint_as_float(u[e] << 16)), fq(__uint_as_float(u[e] & 0xFFFF0000u)));
+            } else {
+                out[2 * c] = g_bf16x2(fq(__uint_as_float(u[0])), fq(__uint_as_float(u[1])));
+                out[2 * c + 1] = g_bf16x2(fq(__uint_as_float(u[2])), fq(__uint_as_float(u[3])));
+            }
+        }
         g_tmem_st16(taddr + 16u * (uint32_t)h, out);
     }
 }
@@ -448,30 +496,40 @@ struct GRing {
 
 // ----------------------------------------------------------------- kernel --
 
+// WM: 0 = packed codes (dequant on load), 1 = bf16 / fp32 weights and clips
+// (fake-quant on load); two instantiations, so that neither pays the
+// other's registers.
+template <int WM>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_dequant_kernel(const __grid_constant__ GemmParams P) {
     extern __shared__ unsigned char g_smem[];
     const uint32_t raw = g_smem_u32(g_smem);
     const uint32_t base = (raw + 1023u) & ~1023u;          // SWIZZLE_128B tiles: 1024-byte aligned
     const int DX = P.dx, DC = P.dc, DW = P.dw, DD = P.dd, NT = P.nt, NI = P.ni, CS = P.cs;
+    const int XS = P.xs, XPC = CS / XS;                    // stages per X slot, X slots per chunk
     const uint32_t xs_bytes = (uint32_t)NT * 128u;         // one stage of X
-    const uint32_t x_bytes = xs_bytes * (uint32_t)CS;      // an X chunk slot
-    const uint32_t cb = P.qbits == 6 ? 48u : 64u;          // code bytes of a row's 64-code stage
-    const uint32_t crow = cb * (uint32_t)CS;               // code bytes of a row's chunk
+    const uint32_t x_bytes = xs_bytes * (uint32_t)XS;      // an X slot
+    // bytes of a row's 64-wide stage in a code slot: packed codes, or the
+    // weights themselves in the weight modes (bf16: one 128-byte swizzled
+    // row; fp32: two 128-byte halves, 16 KB apart)
+    const uint32_t cb = P.wmode == 1 ? 128u : P.wmode == 2 ? 256u : P.qbits == 6 ? 48u : 64u;
+    const uint32_t crow = cb * (uint32_t)CS;               // bytes of a row's chunk
     const uint32_t c_bytes = (uint32_t)kGemmBN * crow;     // a code chunk slot
     // [X ring][code ring][barriers]
     const uint32_t cs0 = base + (uint32_t)DX * x_bytes;
     const uint32_t bars = base + (uint32_t)(kGemmSmemBytes - 1024 - kGemmBarBytes);
     auto full_x = [&](int s) { return bars + 8u * (uint32_t)s; };
-    auto full_c = [&](int s) { return bars + 8u * (uint32_t)(kGemmMaxX + s); };
-    auto empty_c = [&](int s) { return bars + 8u * (uint32_t)(kGemmMaxX + kGemmMaxC + s); };
+    auto x_done = [&](int s) { return bars + 8u * (uint32_t)(kGemmMaxX + s); };   // an X slot's MMAs are done
+    constexpr int kB0 = 2 * kGemmMaxX;
+    auto full_c = [&](int s) { return bars + 8u * (uint32_t)(kB0 + s); };
+    auto empty_c = [&](int s) { return bars + 8u * (uint32_t)(kB0 + kGemmMaxC + s); };
     auto full_w = [&](int s, int k) {                      // sub-stage k of W_hat chunk slot s
-        return bars + 8u * (uint32_t)(kGemmMaxX + 2 * kGemmMaxC + s * kGemmCSMax + k);
+        return bars + 8u * (uint32_t)(kB0 + 2 * kGemmMaxC + s * CS + k);
     };
-    auto done = [&](int s) {                               // a chunk's MMA commit
-        return bars + 8u * (uint32_t)(kGemmMaxX + 2 * kGemmMaxC + kGemmMaxW * kGemmCSMax + s);
+    auto done = [&](int s) {                               // a chunk's MMA commit (frees its W_hat slot)
+        return bars + 8u * (uint32_t)(kB0 + 2 * kGemmMaxC + kGemmMaxWS + s);
     };
     const uint32_t acc_full0 =
-        bars + 8u * (uint32_t)(kGemmMaxX + 2 * kGemmMaxC + kGemmMaxW * kGemmCSMax + kGemmMaxDone);
+        bars + 8u * (uint32_t)(kB0 + 2 * kGemmMaxC + kGemmMaxWS + kGemmMaxDone);
     auto acc_full = [&](int j) { return acc_full0 + 8u * (uint32_t)j; };   // issuer j's segment sums are ready
     const uint32_t acc_empty = acc_full0 + 16u;                             // the epilogue has read them
     const uint32_t fin = acc_full0 + 24u;                                   // 2 barriers: an issuer's MMAs are all done
@@ -484,7 +542,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_dequant_kernel(const __g
     it.init(P);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < DX; ++s) g_bar_init(full_x(s), 1);
+        for (int s = 0; s < DX; ++s) {
+            g_bar_init(full_x(s), 1);
+            g_bar_init(x_done(s), 1);
+        }
         for (int s = 0; s < DC; ++s) {
             g_bar_init(full_c(s), P.code_copy ? 32 : 1);
             g_bar_init(empty_c(s), 4 * CS);                // four warps per sub-stage
@@ -532,7 +593,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_dequant_kernel(const __g
                 ok = false;
                 break;
             }
-            if (!P.code_copy) {
+            if (WM != 0) {
+                // weight modes (one stage per chunk): the stage's 128 x 64
+                // weights, 128-byte swizzled rows; K past the end zero-filled
+                if (lane == 0) {
+                    g_arrive_tx(full_c(rc.s), c_bytes);
+                    const int kx = it.c * kGemmBK;
+                    if (P.wmode == 1) {
+                        g_tma_load_2d(c_tile(rc.s), &P.tmap_w, kx, n0, full_c(rc.s));
+                    } else if (P.w3d) {
+                        g_tma_load_3d(c_tile(rc.s), &P.tmap_w, 0, n0, 2 * it.c, full_c(rc.s));
+                    } else {
+                        g_tma_load_2d(c_tile(rc.s), &P.tmap_w, kx, n0, full_c(rc.s));
+                        g_tma_load_2d(c_tile(rc.s) + 128u * kGemmBN, &P.tmap_w, kx + 32, n0, full_c(rc.s));
+                    }
+                }
+            } else if (!P.code_copy) {
                 if (lane == 0) {
                     g_arrive_tx(full_c(rc.s), c_bytes);    // out-of-range rows / bytes are zero-filled
                     g_tma_load_2d(c_tile(rc.s), &P.tmap_w, it.c * (int)crow, n0, full_c(rc.s));
@@ -563,39 +639,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_dequant_kernel(const __g
             if (!g_wait_warp(full_c((int)(q % DC)), (uint32_t)((q / DC) & 1))) ok = false;
     } else if (warp == 3) {
         // --------------------------------------------------- X producer --
-        GRing rx, rdx;                                     // X slots, the commit of chunk seq - DX
+        GRing rx;                                          // X slots
         rx.init(DX);
-        rdx.init(DD);
         int64_t cur_tile = -1;
         int m0 = 0;
-        int64_t issued = 0;
-        for (; it.valid() && ok; it.next(), rx.next()) {
+        int64_t xseq = 0;                                  // X slots issued
+        for (; it.valid() && ok; it.next()) {
             if (it.tile != cur_tile) {
                 cur_tile = it.tile;
                 m0 = (int)(it.tile % P.tiles_m) * NT;
             }
-            // the slot's previous chunk has been consumed by its MMAs
-            if (it.seq >= DX) {
-                if (!g_wait_warp(done(rdx.s), rdx.ph)) {
+            for (int j = 0; j < XPC && ok; ++j, rx.next(), ++xseq) {
+                // the slot's previous stages have been consumed by their MMAs
+                if (xseq >= DX && !g_wait_warp(x_done(rx.s), rx.ph ^ 1u)) {
                     ok = false;
                     break;
                 }
-                rdx.next();
-            }
-            if (lane == 0) {
-                if (P.x3d) {
-                    g_arrive_tx(full_x(rx.s), x_bytes);    // K stages past the end are zero-filled
-                    g_tma_load_3d(x_tile(rx.s), &P.tmap_x, 0, m0, it.c * CS, full_x(rx.s));
-                } else {
-                    g_arrive_tx(full_x(rx.s), xs_bytes * (uint32_t)(it.hi - it.lo + 1));
-                    for (int k = it.lo; k <= it.hi; ++k)
-                        g_tma_load_2d(x_tile(rx.s) + (uint32_t)k * xs_bytes, &P.tmap_x, (it.c * CS + k) * kGemmBK, m0,
-                                      full_x(rx.s));
+                if (lane == 0) {
+                    const int k0 = j * XS;
+                    if (P.x3d) {
+                        g_arrive_tx(full_x(rx.s), x_bytes);    // K stages past the end are zero-filled
+                        g_tma_load_3d(x_tile(rx.s), &P.tmap_x, 0, m0, it.c * CS + k0, full_x(rx.s));
+                    } else {
+                        const int a = max(k0, it.lo), b = min(k0 + XS - 1, it.hi);
+                        g_arrive_tx(full_x(rx.s), b >= a ? xs_bytes * (uint32_t)(b - a + 1) : 0u);
+                        for (int k = a; k <= b; ++k)
+                            g_tma_load_2d(x_tile(rx.s) + (uint32_t)(k - k0) * xs_bytes, &P.tmap_x,
+                                          (it.c * CS + k) * kGemmBK, m0, full_x(rx.s));
+                    }
                 }
             }
-            issued = it.seq + 1;
         }
-        for (int64_t q = max((int64_t)0, issued - DX); q < issued; ++q)
+        for (int64_t q = max((int64_t)0, xseq - DX); q < xseq; ++q)
             if (!g_wait_warp(full_x((int)(q % DX)), (uint32_t)((q / DX) & 1))) ok = false;
     } else if (warp == 1 || warp == 2) {
         // -------------------------------------------------------- MMA --
@@ -609,32 +684,42 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_dequant_kernel(const __g
             uint32_t seg_ph = 0u;                          // parity of the epilogue's next acc_empty phase
             bool fresh = true;                             // next MMA into acc starts a sum
             int mine = 0;                                  // seq % NI, kept incrementally
-            for (; it.valid() && ok; it.next(), rx.next(), rw.next(), rd.next(), mine = mine + 1 == NI ? 0 : mine + 1) {
+            for (; it.valid() && ok; it.next(), rw.next(), rd.next(), mine = mine + 1 == NI ? 0 : mine + 1) {
                 if (it.seg_first && it.seq > 0) {
                     // a new segment: the epilogue must have read the previous one
                     if (!g_wait_warp(acc_empty, seg_ph)) ok = false;
                     seg_ph ^= 1u;
                     fresh = true;
                 }
-                if (ok && mine == j) {
-                    if (!g_wait_warp(full_x(rx.s), rx.ph)) {
-                        ok = false;
-                        break;
-                    }
-                    for (int k = it.lo; k <= it.hi && ok; ++k) {
-                        if (!g_wait_warp(full_w(rw.s, k), rw.ph)) {
+                if (!ok) break;
+                if (mine != j) {                           // the other issuer's chunk: keep the X ring in step
+                    for (int xj = 0; xj < XPC; ++xj) rx.next();
+                } else {
+                    for (int xj = 0; xj < XPC && ok; ++xj, rx.next()) {
+                        const int k0 = xj * XS, a = max(k0, it.lo), b = min(k0 + XS - 1, it.hi);
+                        // waited even without a stage to run: the slot may be
+                        // refilled only after this copy has landed
+                        if (!g_wait_warp(full_x(rx.s), rx.ph)) {
                             ok = false;
                             break;
                         }
-                        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-                        g_mma_stage_ts(acc, tmem + w_col0 + 32u * (uint32_t)(rw.s * CS + k),
-                                       x_tile(rx.s) + (uint32_t)k * xs_bytes, P.idesc, fresh ? 0u : 1u);
-                        fresh = false;
+                        for (int k = a; k <= b; ++k) {
+                            if (!g_wait_warp(full_w(rw.s, k), rw.ph)) {
+                                ok = false;
+                                break;
+                            }
+                            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                            g_mma_stage_ts(acc, tmem + w_col0 + 32u * (uint32_t)(rw.s * CS + k),
+                                           x_tile(rx.s) + (uint32_t)(k - k0) * xs_bytes, P.idesc, fresh ? 0u : 1u);
+                            fresh = false;
+                        }
+                        if (!ok) break;
+                        g_commit(x_done(rx.s));            // the X slot is free once these MMAs are done
                     }
                     if (!ok) break;
-                    g_commit(done(rd.s));                  // frees the chunk's X slot and W_hat slot
+                    g_commit(done(rd.s));                  // the chunk's W_hat slot likewise
                 }
-                if (ok && it.seg_last) g_commit(acc_full(j)); // the segment's sums (of this issuer) are complete
+                if (it.seg_last) g_commit(acc_full(j));    // the segment's sums (of this issuer) are complete
             }
             g_commit(fin + 8u * (uint32_t)j);
             if (!g_wait_warp(fin + 8u * (uint32_t)j, 0u)) ok = false;
@@ -701,6 +786,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_dequant_kernel(const __g
         int pc = 0;                                        // seq % cpg, kept incrementally
         int64_t cur_tile = -1;
         GDeq deq{};
+        Scale fq{};                                        // weight modes: the row's clip and scale
         for (; it.valid() && ok; it.next(), rc.next(), rw.next(), pc = pc + 1 == cpg ? 0 : pc + 1) {
             const bool reuse = it.seq >= DW;
             const int rd_s = rd.s;
@@ -724,8 +810,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_dequant_kernel(const __g
             if (it.tile != cur_tile) {
                 cur_tile = it.tile;
                 const int64_t n = (it.tile / P.tiles_m) * kGemmBN + r;
-                const float srow = n < P.N ? __half2float(__ushort_as_half(P.scale[n])) : 0.0f;
-                deq = g_deq_consts(P.qbits, srow);
+                if constexpr (WM == 0) {
+                    const float srow = n < P.N ? __half2float(__ushort_as_half(P.scale[n])) : 0.0f;
+                    deq = g_deq_consts(P.qbits, srow);
+                } else {
+                    uint16_t hb;
+                    bool range;
+                    const float c = n < P.N ? P.clip[n] : 0.0f;
+                    fq = make_scale(__float_as_uint(c), P.qbits == 6 ? 31 : 127, P.export_scale != 0, &hb, &range);
+                    if (range && P.status) atomicOr(reinterpret_cast<unsigned int*>(P.status), 0x2u);
+                }
             }
             if (!g_wait_warp(full_c(rc.s), rc.ph)) {
                 ok = false;
@@ -734,8 +828,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_dequant_kernel(const __g
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
             const uint32_t codes = c_tile(rc.s) + (uint32_t)r * crow + (uint32_t)k * cb;
             const uint32_t taddr = lane_addr + 32u * (uint32_t)(rw.s * CS + k);
-            if (P.qbits == 6) g_dequant_stage<6>(codes, taddr, deq);
-            else g_dequant_stage<8>(codes, taddr, deq);
+            if constexpr (WM != 0) {
+                if (P.wmode == 1) g_fakequant_stage<kBF16>(c_tile(rc.s), r, taddr, fq);
+                else g_fakequant_stage<kF32>(c_tile(rc.s), r, taddr, fq);
+            } else {
+                if (P.qbits == 6) g_dequant_stage<6>(codes, taddr, deq);
+                else g_dequant_stage<8>(codes, taddr, deq);
+            }
             asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
             __syncwarp();

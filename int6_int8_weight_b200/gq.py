@@ -41,7 +41,8 @@ STATUS_NAMES = {0: "GQ_OK", 1: "GQ_ERR_INVALID_ARG", 2: "GQ_ERR_UNSUPPORTED",
 EXPORTED = ("gq_row_clip_select", "gq_fakequant_fwd", "gq_fakequant_average", "gq_ste_bwd", "gq_export_pack",
             "gq_export_pack_noalloc", "gq_dequant", "gq_gemm_dequant", "gq_workspace_size", "gq_packed_row_bytes", "gq_k_from_p",
             "gq_plan_kind", "gq_status_string", "gq_last_cuda_error", "gq_last_cuda_error_string",
-            "gq_test_arm_wait_expiry", "gq_gptq_quantize", "gq_gptq_hessian", "gq_gptq_workspace_size")
+            "gq_test_arm_wait_expiry", "gq_gptq_quantize", "gq_gptq_hessian", "gq_gptq_workspace_size",
+            "gq_gemm_fakequant")
 
 
 class GQError(RuntimeError):
@@ -82,9 +83,10 @@ def _load() -> C.CDLL:
     L.gq_ste_bwd.argtypes = [vp, vp, i32, i64, i32, vp]
     L.gq_dequant.argtypes = [vp, vp, i32, i32, i64, i64, vp, i32, vp]
     L.gq_gemm_dequant.argtypes = [vp, i64, i64, i64, vp, vp, i32, i64, vp, i64, vp, vp]
+    L.gq_gemm_fakequant.argtypes = [vp, i64, i64, i64, vp, i32, i64, vp, i32, i32, i64, vp, i64, vp, vp]
     for f in ("gq_row_clip_select", "gq_fakequant_fwd", "gq_fakequant_average", "gq_export_pack",
               "gq_export_pack_noalloc",
-              "gq_ste_bwd", "gq_dequant", "gq_gemm_dequant"):
+              "gq_ste_bwd", "gq_dequant", "gq_gemm_dequant", "gq_gemm_fakequant"):
         getattr(L, f).restype = i32
     L.gq_gptq_quantize.argtypes = [T, vp, f64, vp, sz, vp, vp]
     L.gq_gptq_quantize.restype = i32
@@ -449,6 +451,26 @@ def gptq_quantize(req: Request, H: torch.Tensor, percdamp: float = 0.01, stream=
     if check_status:
         o.status = int(st[0].item())
     return o
+
+
+def gemm_fakequant(x: torch.Tensor, w: torch.Tensor, clip: torch.Tensor, qbits: int = 6,
+                   mode: int = GQ_SCALE_F32, y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Y = X @ W_hat^T with W_hat the fake-quant weight of ``w`` (fp32 / bf16
+    [N, K], rows contiguous) under the row clips ``clip`` (fp32 [N]), built in
+    the GEMM's weight load (tcgen05); binary32 (GQ_SCALE_F32) or binary16
+    (GQ_SCALE_F16) row scales as in gq_fakequant_fwd.  ``x`` is bf16 [M, K]."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a bf16 [M, K] tensor with contiguous rows")
+    if w.dim() != 2 or w.stride(1) != 1 or clip.dtype != torch.float32 or not clip.is_contiguous():
+        raise ValueError("w must be [N, K] with contiguous rows and clip a contiguous fp32 [N] tensor")
+    M, K = x.shape
+    N = w.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    _check(LIB.gq_gemm_fakequant(x.data_ptr(), M, K, x.stride(0), w.data_ptr(), _dtype_code(w), w.stride(0),
+                                 clip.data_ptr(), qbits, mode, N, y.data_ptr(), y.stride(0), None,
+                                 _stream(stream)), "gq_gemm_fakequant")
+    return y
 
 
 def ste_bwd(g_out: torch.Tensor, g_w: torch.Tensor | None = None, stream=None) -> torch.Tensor:

@@ -182,11 +182,11 @@ def test_gemm_argument_errors_before_launch(gq):
         (dict(i=1, v=-1), 1),           # M < 0
         (dict(i=3, v=32), 1),           # ldx < K
         (dict(i=9, v=4), 1),            # ldy < N
-        (dict(i=2, v=48, j=3, w=48), 2),  # K not a multiple of 64
+        (dict(i=2, v=50, j=3, w=56), 2),  # int6 rows of 39 bytes: neither TMA nor 4-byte copies
         (dict(i=0, v=X + 2), 3),        # activations not 16-byte aligned
-        (dict(i=4, v=P + 8), 3),        # packed codes not 16-byte aligned
-        (dict(i=8, v=Y + 4), 3),        # Y not 16-byte aligned
-        (dict(i=9, v=10), 3),           # ldy % 4 != 0
+        (dict(i=3, v=68), 3),           # activation pitch not a multiple of 8
+        (dict(i=4, v=P + 8), 3),        # packed codes (48-byte rows) not 16-byte aligned
+        (dict(i=8, v=Y + 2), 3),        # Y not 4-byte aligned
         (dict(i=0, v=0), 1),            # null activations
     ]
     for case, code in bad_cases:
@@ -205,3 +205,18 @@ def test_wait_expiry_hook_rejects_bad_arguments(gq):
     assert gq.LIB.gq_test_arm_wait_expiry(-1, 5_000_000) == 1
     assert gq.LIB.gq_test_arm_wait_expiry(0, 999_999) == 1
     assert gq.LIB.gq_test_arm_wait_expiry(0, 4_000_000_001) == 1
+
+
+def test_gemm_fakequant_argument_errors_before_launch(gq):
+    """gq_gemm_fakequant likewise (fake device addresses never dereferenced)."""
+    L = gq.LIB
+    X, W, C, Y = 0x100000, 0x200000, 0x300000, 0x400000
+    ok = [X, 4, 64, 64, W, 0, 64, C, 6, 0, 8, Y, 8, None, None]
+    for i, v, code in ((5, 2, 1), (9, 5, 1), (8, 4, 1), (6, 32, 1), (10, -1, 1), (4, W + 4, 3), (6, 66, 3),
+                       (7, C + 2, 3), (7, 0, 1), (0, X + 8, 3)):
+        args = list(ok)
+        args[i] = v
+        assert L.gq_gemm_fakequant(*args) == code, (i, v, code)
+    empty = list(ok)
+    empty[1] = 0
+    assert L.gq_gemm_fakequant(*empty) == 0

@@ -1,4 +1,6 @@
-"""GPU parity of the dequant-on-load GEMM (gq_gemm_dequant) against the oracle.
+"""GPU parity of the consuming GEMMs against the oracle: gq_gemm_dequant (the
+weight rebuilt from packed codes) and gq_gemm_fakequant (fake-quantized from
+fp32 / bf16 weights and row clips in the weight load).
 
 Y = X @ W_hat^T where W_hat[n, k] = bf16(RN(q[n, k] * s[n])) comes from the
 packed codes and binary16 scales.  The reference is oracle/gemm.py: W_hat
@@ -154,3 +156,64 @@ def test_gemm_dequant_fresh_inputs(gq, qbits):
     for M, N, K in ((128, 256, 512), (256, 256, 512), (300, 384, 2048), (16, 512, 4096)):
         for rep in range(3):
             _case(gq, M, N, K, qbits, seed=1000 * rep + M + N + K + qbits)
+
+
+@pytest.mark.parametrize("wdt", ["f32", "bf16"])
+@pytest.mark.parametrize("M,N,K,qbits,mode,p", [
+    (16, 1584, 528, 6, 0, 1.0),       # the 11-layer model's unified projection, training scales
+    (64, 528, 1584, 6, 0, 1.0),       # its MLP down projection
+    (100, 256, 1000, 8, 1, 0.999),    # binary16 scales, percentile clip, ragged K
+    (300, 384, 2048, 6, 1, 0.9999),   # two 256-token tiles
+    (1, 128, 40, 6, 0, 1.0),          # K shorter than a stage
+    (1024, 16384, 128, 6, 0, 1.0),    # whole tiles
+])
+def test_gemm_fakequant_matches_oracle(gq, wdt, M, N, K, qbits, mode, p):
+    """W_hat is the fake-quant output of gq_fakequant_fwd for the same weight
+    (rounded to bf16 for fp32 weights); the clips come from the library's own
+    select and must equal the oracle's."""
+    rng = np.random.default_rng(M + N + K + qbits)
+    w = synth.random_matrix(rng, N, K, "t3")
+    if wdt == "bf16":
+        w = synth.to_bf16_bits(w).reshape(N, K)
+        W = torch.from_numpy(w.view(np.int16).copy()).cuda().view(torch.bfloat16)
+    else:
+        W = torch.from_numpy(w).cuda()
+    (c,) = gq.row_clip_select([gq.Request(W, qbits, p)])
+    x = _x(rng, M, K)
+    X = torch.from_numpy(x.view(np.int16).copy()).cuda().view(torch.bfloat16)
+    ldy = N + 1
+    Ypad = torch.full((M, ldy), 7.0, device="cuda")
+    st = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    rc = gq.LIB.gq_gemm_fakequant(X.data_ptr(), M, K, K, W.data_ptr(), 1 if wdt == "bf16" else 0, K,
+                                  c.clip.data_ptr(), qbits, mode, N, Ypad.data_ptr(), ldy, st.data_ptr(), None)
+    torch.cuda.synchronize()
+    assert rc == 0 and int(st[0]) == 0, (rc, int(st[0]))
+    assert bool((Ypad[:, N:] == 7.0).all())
+    ref = oracle.quantize(w, qbits, p, export=mode == 1)
+    assert ref.status == oracle.OR_OK
+    assert np.array_equal(c.clip.cpu().numpy().view(np.uint32), ref.clip.view(np.uint32))
+    w_hat = ref.dq if wdt == "bf16" else oracle.f32_to_bf16_bits(ref.dq).reshape(N, K)
+    y_ref, a = GM.contraction(x, w_hat)
+    got = Ypad[:, :N].cpu().numpy().astype(np.float64)
+    bad = np.argwhere(np.abs(got - y_ref) > _bound(K, a))
+    assert bad.size == 0, (f"{wdt} M{M} N{N} K{K}: {len(bad)} outside the bound, first {tuple(bad[0])}: "
+                           f"got {got[tuple(bad[0])]!r} want {y_ref[tuple(bad[0])]!r}")
+
+
+def test_gemm_fakequant_errors(gq):
+    X = torch.zeros(4, 64, dtype=torch.bfloat16, device="cuda")
+    W = torch.zeros(8, 64, device="cuda")
+    clip = torch.ones(8, device="cuda")
+    Y = torch.empty(4, 8, device="cuda")
+    L = gq.LIB
+    args = [X.data_ptr(), 4, 64, 64, W.data_ptr(), 0, 64, clip.data_ptr(), 6, 0, 8, Y.data_ptr(), 8, None, None]
+    assert L.gq_gemm_fakequant(*args) == 0
+    bad = list(args); bad[5] = 3                          # weight dtype
+    assert L.gq_gemm_fakequant(*bad) == 1
+    bad = list(args); bad[9] = 2                          # scale mode
+    assert L.gq_gemm_fakequant(*bad) == 1
+    bad = list(args); bad[6] = 62                         # weight pitch: not a multiple of 16 bytes
+    assert L.gq_gemm_fakequant(*bad) in (1, 3)
+    bad = list(args); bad[7] = None                       # no clips
+    assert L.gq_gemm_fakequant(*bad) == 1
+    torch.cuda.synchronize()
