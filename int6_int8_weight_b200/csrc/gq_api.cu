@@ -25,7 +25,6 @@ namespace {
 using namespace gq;
 
 constexpr size_t kWsSlot = 8448;      // 2048 x u32 histogram + 16 x u32 state, 256-aligned
-constexpr int64_t kWaveBytes = 48ll << 20;   // per-tensor inputs per wave (L2 is 126 MB)
 constexpr int kMaxDevices = 64;
 std::atomic<int> g_sm_count[kMaxDevices];
 
@@ -373,13 +372,6 @@ gq_status quantize_batch(const gq_tensor* t, int n, Op op, bool f16_mode, void* 
     std::vector<RowDesc> rows_w, rows_c;   // warp teams / block teams
     std::vector<RowDesc> rows_tma;         // pipelined through shared memory
     std::vector<PassDesc> pass;
-    // per-tensor groups, in waves whose inputs fit in L2 together
-    struct Wave {
-        std::vector<SelDesc> sel;
-        std::vector<RowDesc> tma, w, c;
-        int64_t bytes = 0;
-    };
-    std::vector<Wave> waves;
     size_t slot = 0;
     for (int i = 0; i < n; ++i) {
         const gq_tensor& T = t[i];
@@ -462,41 +454,19 @@ gq_status quantize_batch(const gq_tensor* t, int n, Op op, bool f16_mode, void* 
             D.items = T.rows;
         }
         D.flags = flags;
-        std::vector<RowDesc>* tma = &rows_tma;
-        std::vector<RowDesc>* wt = &rows_w;
-        std::vector<RowDesc>* ct = &rows_c;
-        if (T.gran == GQ_PER_TENSOR) {
-            // a per-tensor group reads its tensor four times (three histogram
-            // passes, then the quantize pass): group the tensors in waves of
-            // at most kWaveBytes of input so that the later passes of a wave
-            // find its tensors in L2
-            const int64_t bytes = T.rows * T.cols * esz;
-            if (waves.empty() || (waves.back().bytes > 0 && waves.back().bytes + bytes > kWaveBytes))
-                waves.emplace_back();
-            Wave& Wv = waves.back();
-            Wv.bytes += bytes;
-            Wv.sel.push_back(sel.back());
-            sel.pop_back();
-            tma = &Wv.tma;
-            wt = &Wv.w;
-            ct = &Wv.c;
-        }
         // column scales read as float4 by the pipelined kernel (else the row kernels)
         if (tma_eligible(T, flags) && (!T.col_scale || (flags & kVecCol)))
-            tma->push_back(D);
+            rows_tma.push_back(D);
         else if (T.cols <= 2048)
-            wt->push_back(D);
+            rows_w.push_back(D);
         else
-            ct->push_back(D);
+            rows_c.push_back(D);
     }
 
-    gq_status st = GQ_OK;
-    for (Wave& Wv : waves) {
-        if ((st = run_per_tensor_select(Wv.sel, stream)) != GQ_OK) return st;
-        if ((st = run_rows_tma(Wv.tma, stream)) != GQ_OK) return st;
-        if ((st = run_rows<1>(Wv.w, stream)) != GQ_OK) return st;
-        if ((st = run_rows<kBlockWarps>(Wv.c, stream)) != GQ_OK) return st;
-    }
+    // the per-tensor clips first (three streaming passes over those tensors),
+    // then every row pass
+    gq_status st = run_per_tensor_select(sel, stream);
+    if (st != GQ_OK) return st;
     st = run_rows_tma(rows_tma, stream);
     if (st != GQ_OK) return st;
     st = run_rows<1>(rows_w, stream);

@@ -247,6 +247,12 @@ __device__ __forceinline__ void g_tmem_st16(uint32_t taddr, const uint32_t (&v)[
         : "memory");
 }
 
+__device__ __forceinline__ void g_tmem_st8(uint32_t taddr, const uint32_t (&v)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+                 "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+                 : "memory");
+}
+
 __device__ __forceinline__ void g_tmem_ld16(uint32_t taddr, float (&f)[16]) {
     uint32_t v[16];
     asm volatile(
@@ -378,39 +384,129 @@ __device__ __forceinline__ void g_dequant_stage(uint32_t codes, uint32_t taddr, 
     }
 }
 
+// Per-row constants of the fake-quant in the load.  The paired path below
+// drops the clip to +-c and keeps only the clamp to +-qmax: for |w| <= c the
+// clip does nothing, and for |w| > c both give +-qmax exactly when the
+// row's own clip value lands there, RN(c / s) >= qmax (true for every
+// binary32 scale and every normal binary16 one; a coarse binary16
+// subnormal scale can break it).  Rows where this fails, or whose scale has
+// no normal reciprocal, take the per-element path.
+struct GFq {
+    Scale S;
+    bool paired;
+};
+
+__device__ __forceinline__ GFq g_fq_consts(const Scale& S) {
+    GFq f;
+    f.S = S;
+    f.paired = false;
+    if (S.fast && !S.zero) {
+        const float t = __fdiv_rn(S.c, S.s);                       // < 256 for any scale make_scale gives
+        const float q = __fsub_rn(__fadd_rn(t, kMagic), kMagic);   // round half to even
+        f.paired = q >= S.qmaxf;
+    }
+    return f;
+}
+
+// The paired constants: (rcp, rcp), (kMagic, kMagic), (s, s).
+struct GFq2 {
+    uint64_t r2, m2, s2;
+    float lo, hi;                // kMagic -+ qmax
+};
+
+// Two weights -> one bf16x2 word of W_hat on the paired path, and the larger
+// distance of their scaled values from the rounded ones (the guard of the
+// reciprocal quotient, as in the row kernel: at most 0.5 - 2^-13 means both
+// codes are round_half_even(RN(w / s)), whether or not the code generator
+// fuses the product into the sums; beyond it the caller redoes the weights
+// with the exact division).  |w / s| >= 256 clamps to +-qmax on either side.
+__device__ __forceinline__ uint32_t g_fq_pair(float w0, float w1, const GFq2& f, float& dmax) {
+    uint64_t Y, B, N, E;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(Y) : "l"(g_f2(w0, w1)), "l"(f.r2));
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(B) : "l"(Y), "l"(f.m2));
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(N) : "l"(B), "l"(f.m2));
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(E) : "l"(Y), "l"(N));
+    float e0, e1, b0, b1;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(e0), "=f"(e1) : "l"(E));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(b0), "=f"(b1) : "l"(B));
+    dmax = fmaxf(dmax, fmaxf(fabsf(e0), fabsf(e1)));
+    b0 = fminf(fmaxf(b0, f.lo), f.hi);
+    b1 = fminf(fmaxf(b1, f.lo), f.hi);
+    // w_hat = RN((b - kMagic) * s): the difference q is exact
+    uint64_t Q, D;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(Q) : "l"(g_f2(b0, b1)), "l"(f.m2));
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(D) : "l"(Q), "l"(f.s2));
+    float d0, d1;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(D));
+    return g_bf16x2(d0, d1);
+}
+
 // One weight row's 64-wide stage, fake-quantized on the way into TMEM:
 // w_hat = RN(q * s) with q = clamp(round_half_even(clip(w, -c, c) / s)), the
 // very arithmetic of the fused row kernel (quantize_offset / offset_to_dq),
 // then rounded to bf16 for the tensor cores.  The stage sits in shared
 // memory as 128-byte rows with the 128-byte swizzle (16-byte chunk j of row r
 // at chunk position j ^ (r & 7)): one row of 64 bf16, or two rows of 32 fp32
-// in halves 16 KB apart.
+// in halves 16 KB apart.  Each group of 16 weights takes the paired path
+// when the row allows it and redoes itself per element if its guard trips.
 template <int DT>
-__device__ __forceinline__ void g_fakequant_stage(uint32_t tile, int r, uint32_t taddr, const Scale& S) {
+__device__ __forceinline__ void g_fakequant_stage(uint32_t tile, int r, uint32_t taddr, const GFq& f) {
     const uint32_t sw = (uint32_t)(r & 7), row = tile + 128u * (uint32_t)r;
-    auto fq = [&](float w) { return offset_to_dq(quantize_offset(w, S), S); };
+    auto fq = [&](float w) { return offset_to_dq(quantize_offset(w, f.S), f.S); };
+    // 16-byte chunk c (0 .. 7) of the row's stage: 8 bf16 or 4 fp32 weights
+    auto chunk = [&](int c, uint32_t (&u)[4]) {
+        const uint32_t j = DT == kBF16 ? (uint32_t)c : (uint32_t)(c & 7);
+        const uint32_t src = (DT == kBF16 ? row : row + (uint32_t)(c >> 3) * 128u * kGemmBN) + ((j ^ sw) << 4);
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3])
+                     : "r"(src)
+                     : "memory");
+    };
+    GFq2 f2;
+    f2.r2 = g_f2(f.S.rcp, f.S.rcp);
+    f2.m2 = g_f2(kMagic, kMagic);
+    f2.s2 = g_f2(f.S.s, f.S.s);
+    f2.lo = kMagic - f.S.qmaxf;
+    f2.hi = kMagic + f.S.qmaxf;
+    constexpr int kChunks = DT == kBF16 ? 2 : 4;           // chunks per 16 weights
+#pragma unroll 1
+    for (int g = 0; g < 4; ++g) {                          // 16 weights -> 8 bf16x2 columns
+        uint32_t out[8];
+        bool exact = !f.paired;
+        if (f.paired) {
+            float dmax = 0.0f;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {                          // 32 weights -> 16 bf16x2 columns
-        uint32_t out[16];
+            for (int c = 0; c < kChunks; ++c) {
+                uint32_t u[4];
+                chunk(kChunks * g + c, u);
+                if constexpr (DT == kBF16) {
 #pragma unroll
-        for (int c = 0; c < (DT == kBF16 ? 4 : 8); ++c) {
-            uint32_t u[4];
-            const uint32_t j = DT == kBF16 ? (uint32_t)(4 * h + c) : (uint32_t)c;
-            const uint32_t src = (DT == kBF16 ? row : row + (uint32_t)h * 128u * kGemmBN) + ((j ^ sw) << 4);
-            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3])
-                         : "r"(src)
-                         : "memory");
-            if constexpr (DT == kBF16) {
+                    for (int e = 0; e < 4; ++e)
+                        out[4 * c + e] = g_fq_pair(__uint_as_float(u[e] << 16), __uint_as_float(u[e] & 0xFFFF0000u),
+                                                   f2, dmax);
+                } else {
+                    out[2 * c] = g_fq_pair(__uint_as_float(u[0]), __uint_as_float(u[1]), f2, dmax);
+                    out[2 * c + 1] = g_fq_pair(__uint_as_float(u[2]), __uint_as_float(u[3]), f2, dmax);
+                }
+            }
+            exact = dmax > kNearHalf;
+        }
+        if (exact) {
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    out[4 * c + e] = g_bf16x2(fq(__uint_as_float(u[e] << 16)), fq(__uint_as_float(u[e] & 0xFFFF0000u)));
-            } else {
-                out[2 * c] = g_bf16x2(fq(__uint_as_float(u[0])), fq(__uint_as_float(u[1])));
-                out[2 * c + 1] = g_bf16x2(fq(__uint_as_float(u[2])), fq(__uint_as_float(u[3])));
+            for (int c = 0; c < kChunks; ++c) {
+                uint32_t u[4];
+                chunk(kChunks * g + c, u);
+                if constexpr (DT == kBF16) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        out[4 * c + e] = g_bf16x2(fq(__uint_as_float(u[e] << 16)), fq(__uint_as_float(u[e] & 0xFFFF0000u)));
+                } else {
+                    out[2 * c] = g_bf16x2(fq(__uint_as_float(u[0])), fq(__uint_as_float(u[1])));
+                    out[2 * c + 1] = g_bf16x2(fq(__uint_as_float(u[2])), fq(__uint_as_float(u[3])));
+                }
             }
         }
-        g_tmem_st16(taddr + 16u * (uint32_t)h, out);
+        g_tmem_st8(taddr + 8u * (uint32_t)g, out);
     }
 }
 
@@ -786,7 +882,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_dequant_kernel(const __g
         int pc = 0;                                        // seq % cpg, kept incrementally
         int64_t cur_tile = -1;
         GDeq deq{};
-        Scale fq{};                                        // weight modes: the row's clip and scale
+        GFq fq{};                                          // weight modes: the row's clip and scale
         for (; it.valid() && ok; it.next(), rc.next(), rw.next(), pc = pc + 1 == cpg ? 0 : pc + 1) {
             const bool reuse = it.seq >= DW;
             const int rd_s = rd.s;
@@ -817,7 +913,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_dequant_kernel(const __g
                     uint16_t hb;
                     bool range;
                     const float c = n < P.N ? P.clip[n] : 0.0f;
-                    fq = make_scale(__float_as_uint(c), P.qbits == 6 ? 31 : 127, P.export_scale != 0, &hb, &range);
+                    fq = g_fq_consts(make_scale(__float_as_uint(c), P.qbits == 6 ? 31 : 127, P.export_scale != 0,
+                                                &hb, &range));
                     if (range && P.status) atomicOr(reinterpret_cast<unsigned int*>(P.status), 0x2u);
                 }
             }
