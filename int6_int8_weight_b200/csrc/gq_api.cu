@@ -16,6 +16,7 @@
 
 #include "gq_aux_kernels.cuh"
 #include "gq_gemm.cuh"
+#include "gq_gemm_decode.cuh"
 #include "gq_gptq.cuh"
 #include "gq_kernels.cuh"
 #include "gq_rowquant_tma.cuh"
@@ -480,6 +481,7 @@ gq_status quantize_batch(const gq_tensor* t, int n, Op op, bool f16_mode, void* 
 
 std::atomic<void*> g_encode_tiled{nullptr};
 std::atomic<int> g_gemm_smem_set[2][kMaxDevices];
+std::atomic<int> g_dec_smem_set[2][kMaxDevices];
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no
 // link-time dependency on the driver library).
@@ -571,6 +573,54 @@ struct GemmIn {
     const float* clip;
     int export_scale;
 };
+
+// Decode-sized batches (M <= 16) of the dequant-on-load GEMM whose packed
+// rows suit TMA: the register-level kernel of gq_gemm_decode.cuh over units
+// of 256 weight rows x 512 of K, one block per SM; Y is zeroed first (the
+// units add into it).
+gq_status gemm_decode_launch(const void* d_x, int64_t M, int64_t K, int64_t ldx, const uint8_t* d_packed,
+                             const uint16_t* d_scale_f16, int qbits, int64_t prb, int64_t N, float* d_y,
+                             int64_t ldy, int32_t* d_status, cudaStream_t stream) {
+    PFN_cuTensorMapEncodeTiled enc = encode_tiled();
+    if (!enc) return GQ_ERR_UNSUPPORTED;
+    DecParams P;
+    std::memset(&P, 0, sizeof(P));
+    const cuuint64_t gdim[2] = {(cuuint64_t)prb, (cuuint64_t)N};
+    const cuuint64_t gstride[1] = {(cuuint64_t)prb};
+    const cuuint32_t box[2] = {(cuuint32_t)(qbits == 6 ? dec_ss_bytes<6>() : dec_ss_bytes<8>()), 16u};
+    const cuuint32_t estride[2] = {1, 1};
+    if (enc(&P.tmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(d_packed), gdim, gstride, box, estride,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return GQ_ERR_UNSUPPORTED;
+    P.x = static_cast<const uint16_t*>(d_x);
+    P.scale = d_scale_f16;
+    P.y = d_y;
+    P.status = d_status;
+    P.ldx = ldx;
+    P.ldy = ldy;
+    P.M = M;
+    P.N = N;
+    P.K = K;
+    P.kunits = (K + kDecKc - 1) / kDecKc;
+    P.units = ((N + kDecRows - 1) / kDecRows) * P.kunits;
+    const int64_t grid = std::min<int64_t>(sm_count(), P.units);
+    if (cuda_status(cudaMemset2DAsync(d_y, (size_t)ldy * 4, 0, (size_t)N * 4, (size_t)M, stream)) != GQ_OK)
+        return GQ_ERR_CUDA;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GQ_ERR_CUDA;
+    const int qi = qbits == 6 ? 0 : 1;
+    const int smem = qi ? dec_smem_bytes<8>() : dec_smem_bytes<6>();
+    if (dev >= 0 && dev < kMaxDevices && g_dec_smem_set[qi][dev].load() < smem) {
+        if (cuda_status(cudaFuncSetAttribute(qi ? gemm_decode_kernel<8> : gemm_decode_kernel<6>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != GQ_OK)
+            return GQ_ERR_CUDA;
+        g_dec_smem_set[qi][dev].store(smem);
+    }
+    if (qi == 0) gemm_decode_kernel<6><<<(unsigned)grid, kDecThreads, smem, stream>>>(P);
+    else gemm_decode_kernel<8><<<(unsigned)grid, kDecThreads, smem, stream>>>(P);
+    return launch_status();
+}
 
 // The launch shared by the dequant-on-load and the fake-quant-on-load GEMM
 // (arguments already checked).
@@ -934,6 +984,8 @@ gq_status gq_gemm_dequant(const void* d_x, int64_t M, int64_t K, int64_t ldx, co
         return GQ_ERR_MISALIGNED;
     if (K == 0)
         return cuda_status(cudaMemset2DAsync(d_y, (size_t)ldy * 4, 0, (size_t)N * 4, (size_t)M, stream));
+    if (M <= kDecMaxM && tma_codes)
+        return gemm_decode_launch(d_x, M, K, ldx, d_packed, d_scale_f16, qbits, prb, N, d_y, ldy, d_status, stream);
     GemmIn in{};
     in.x = d_x; in.M = M; in.K = K; in.ldx = ldx; in.N = N; in.y = d_y; in.ldy = ldy; in.status = d_status;
     in.stream = stream; in.qbits = qbits; in.wmode = 0; in.packed = d_packed; in.scale = d_scale_f16;

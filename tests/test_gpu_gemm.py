@@ -217,3 +217,62 @@ def test_gemm_fakequant_errors(gq):
     bad = list(args); bad[7] = None                       # no clips
     assert L.gq_gemm_fakequant(*bad) == 1
     torch.cuda.synchronize()
+
+
+# Decode-sized batches (M <= 16) take the register-level kernel
+# (gq_gemm_decode.cuh): units of 256 weight rows x 512 of K, K permuted alike
+# in X and W_hat inside each 64-wide stage, partial sums added into Y.
+@pytest.mark.parametrize("qbits", [6, 8])
+@pytest.mark.parametrize("M,N,K", [
+    (1, 8, 64),           # one 8-row column group, one stage
+    (2, 1000, 512),       # ragged row block, one K unit
+    (7, 257, 1024),       # one row past a row block
+    (9, 4104, 2048),      # N % 256 = 8
+    (15, 300, 528),       # K past the first unit by 16 (a short last stage)
+    (16, 1584, 528),      # the 11-layer model's unified projection
+    (16, 528, 1584),      # its MLP-down projection
+    (3, 100, 16),         # a single 16-wide slice of a stage
+    (16, 2048, 5120),     # ten K units per row block
+])
+def test_gemm_decode_matches_oracle(gq, M, N, K, qbits):
+    _case(gq, M, N, K, qbits, seed=M * 11 + N + K + qbits)
+
+
+@pytest.mark.parametrize("M", [16, 5])
+def test_gemm_decode_unit_runs_sampled(gq, M):
+    """Many units per block, whose runs cross row blocks (flushes in the
+    middle of a run): sampled entries against exactly rounded sums."""
+    N, K, qbits = 8192, 16384, 6
+    rng = np.random.default_rng(M + 5)
+    prb = 3 * ((K + 3) // 4)
+    packed = synth.random_packed_codes(rng, N, prb)
+    scale = synth.random_f16_scales(rng, N)
+    x = _x(rng, M, K)
+    Y = _run(gq, x, packed, scale, qbits, N, K)
+    ms = np.concatenate([[0, M - 1, 0, M - 1], rng.integers(0, M, 2048)])
+    ns = np.concatenate([[0, 0, N - 1, N - 1], rng.integers(0, N, 2048)])
+    rows = np.unique(ns)
+    w = GM.w_hat_bf16(packed[rows], scale[rows], qbits, len(rows), K)
+    where = {int(n): i for i, n in enumerate(rows)}
+    ye, a = GM.contraction_exact(x, w, [(int(m), where[int(n)]) for m, n in zip(ms, ns)])
+    got = Y.cpu().numpy().astype(np.float64)[ms, ns]
+    bad = np.nonzero(np.abs(got - ye) > _bound(K, a))[0]
+    assert bad.size == 0, (M, len(bad), int(ms[bad[0]]), int(ns[bad[0]]), got[bad[0]], ye[bad[0]])
+
+
+def test_gemm_decode_activation_pitch(gq):
+    """X rows wider than K (ldx = K + 24): only the first K columns count."""
+    M, N, K, qbits = 12, 640, 1024, 6
+    rng = np.random.default_rng(9)
+    ref = oracle.quantize(synth.random_matrix(rng, N, K, "t3"), qbits, 1.0, export=True)
+    xw = _x(rng, M, K + 24)
+    X = torch.from_numpy(xw.view(np.int16).copy()).cuda().view(torch.bfloat16)
+    P = torch.from_numpy(ref.packed).cuda()
+    S = torch.from_numpy(ref.scale_f16.view(np.int16).copy()).cuda().view(torch.float16)
+    Y = torch.empty(M, N, device="cuda")
+    assert gq.LIB.gq_gemm_dequant(X.data_ptr(), M, K, K + 24, P.data_ptr(), S.data_ptr(), qbits, N,
+                                  Y.data_ptr(), N, None, None) == 0
+    torch.cuda.synchronize()
+    y_ref, a = GM.contraction(np.ascontiguousarray(xw[:, :K]), GM.w_hat_bf16(ref.packed, ref.scale_f16, qbits, N, K))
+    got = Y.cpu().numpy().astype(np.float64)
+    assert (np.abs(got - y_ref) <= _bound(K, a)).all()
