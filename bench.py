@@ -647,8 +647,7 @@ def gptq_rows(gq, device, out, record):
     fl_h = sum(2 * 2048 * s.shape[1] ** 2 / 2 for (s, _, _, _) in items)
 
     def run_all():
-        for r, H in zip(reqs, Hs):
-            gq.gptq_quantize(r, H, check_status=False)
+        gq.gptq_quantize_batch(reqs, Hs, check_status=False)
 
     def hess_all():
         for (_, _, _, X), H in zip(items, Hs):
@@ -656,7 +655,8 @@ def gptq_rows(gq, device, out, record):
 
     for name, fn, flops, note in (
             ("gptq unified11 export (44 weights, int6 per row)", run_all, fl,
-             "binary64 recurrence + Cholesky, Hessians given; packed int6 + fp16 scales"),
+             "one gq_gptq_quantize_batch call: binary64 recurrence + Cholesky, Hessians given; "
+             "packed int6 + fp16 scales"),
             ("gptq unified11 Hessians (2048 input rows each)", hess_all, fl_h, "H = 2 X^T X in binary64")):
         t = statistics.median(_time_reps(fn, 5))
         tf = flops / t / 1e12

@@ -265,11 +265,9 @@ GQ_API gq_status gq_export_pack(const gq_tensor* t, int n, void* d_ws,
  *
  *  - At most GQ_NOALLOC_MAX_PER_TENSOR per-tensor descriptors per call; a
  *    larger batch returns GQ_ERR_WORKSPACE before anything is launched.
- *  - The first call on a device looks up the array's device address (with
- *    that device current) and caches it until the process exits; make that
- *    first call before any stream capture.  cudaDeviceReset unloads the
- *    library's device code, which makes the cached address stale: do not
- *    call this entry point on a device after resetting it.
+ *  - Every call looks up the array's device address in the current context
+ *    (cudaGetSymbolAddress, no allocation), so it stays valid after a
+ *    cudaDeviceReset reloads the library's device code.
  *  - All calls on a device share the one array and each call clears the part
  *    it uses; calls whose work overlaps on the GPU (different streams, or
  *    different host threads without ordering) race on it.
@@ -381,6 +379,26 @@ GQ_API gq_status gq_test_arm_wait_expiry(int64_t tile, uint64_t wait_ns);
 GQ_API size_t gq_gptq_workspace_size(int64_t rows, int64_t cols);
 GQ_API gq_status gq_gptq_quantize(const gq_tensor* t, const double* d_H, double percdamp, void* d_ws,
                                   size_t ws_bytes, int32_t* d_status, cudaStream_t stream);
+
+/*
+ * GPTQ-lite of n weights in one call: the same computation and outputs as n
+ * calls of gq_gptq_quantize (bitwise), but every step runs once for all the
+ * weights (their chains are independent), so the launches are about
+ * 2 * max(cols) / 64 + 5 per group of 64 weights instead of per weight.
+ *
+ *   t       [n] host array of descriptors, each as for gq_gptq_quantize
+ *   d_H     [n] host array of device pointers: d_H[i] is the fp64 [cols_i,
+ *           cols_i] Hessian of weight i (unused for an empty weight)
+ *   d_ws    device workspace of at least gq_gptq_batch_workspace_size(t, n)
+ *           bytes, 256-byte aligned; weight i takes the
+ *           gq_gptq_workspace_size(rows_i, cols_i) bytes after those of the
+ *           weights before it
+ *   d_status  nullable, [n] int32: d_status[i] reports weight i
+ * Errors as gq_gptq_quantize, checked for every weight before any launch.
+ */
+GQ_API size_t gq_gptq_batch_workspace_size(const gq_tensor* t, int n);
+GQ_API gq_status gq_gptq_quantize_batch(const gq_tensor* t, int n, const double* const* d_H, double percdamp,
+                                        void* d_ws, size_t ws_bytes, int32_t* d_status, cudaStream_t stream);
 
 /*
  * The Hessian of GPTQ-lite from calibration inputs: H = 2 X^T X (accumulate =

@@ -502,20 +502,14 @@ PFN_cuTensorMapEncodeTiled encode_tiled() {
 constexpr size_t kNoAllocSlots = 64;                       // per-tensor groups per call
 constexpr size_t kNoAllocBytes = kNoAllocSlots * kWsSlot;  // 528 KiB per device
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
-std::atomic<void*> g_noalloc_addr[kMaxDevices];
 
-// Device address of g_noalloc_scratch on the current device.  Host code sees
-// only a host-side stand-in for the array, so the address is looked up once
-// per device (with that device current) and cached.
+// Device address of g_noalloc_scratch in the current context.  Host code
+// sees only a host-side stand-in for the array, so the address is looked up
+// on every call: after a device reset or in another context the module is
+// loaded again and an address kept from before would be stale.
 gq_status noalloc_scratch(void** out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return GQ_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return GQ_ERR_UNSUPPORTED;
-    void* p = g_noalloc_addr[dev].load(std::memory_order_acquire);
-    if (!p) {
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return GQ_ERR_CUDA;
-        g_noalloc_addr[dev].store(p, std::memory_order_release);
-    }
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return GQ_ERR_CUDA;
     *out = p;
     return GQ_OK;
 }
@@ -709,10 +703,13 @@ gq_status gemm_launch(const GemmIn& in) {
                 return GQ_ERR_UNSUPPORTED;
         }
     } else if (tma_codes) {
-        const cuuint64_t wdim[2] = {(cuuint64_t)prb, (cuuint64_t)N};
-        const cuuint64_t wstride[1] = {(cuuint64_t)prb};
-        const cuuint32_t wbox[2] = {(cuuint32_t)crow, (cuuint32_t)kGemmBN};
-        if (enc(&P.tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(d_packed), wdim, wstride, wbox,
+        // packed rows as {16 bytes, prb / 16 chunks, N rows}; a copy takes one
+        // chunk more than the row's stages hold, which pads the rows in shared
+        // memory to an odd number of chunks (no bank conflicts)
+        const cuuint64_t wdim[3] = {16, (cuuint64_t)(prb / 16), (cuuint64_t)N};
+        const cuuint64_t wstride[2] = {16, (cuuint64_t)prb};
+        const cuuint32_t wbox[3] = {16, (cuuint32_t)(crow / 16 + 1), (cuuint32_t)kGemmBN};
+        if (enc(&P.tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(d_packed), wdim, wstride, wbox,
                 estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return GQ_ERR_UNSUPPORTED;
@@ -744,7 +741,7 @@ gq_status gemm_launch(const GemmIn& in) {
     // is left, W_hat in the TMEM columns after the accumulators; the commit
     // ring is a multiple of the W_hat depth and at least the X depth (a
     // waiter on any of these barriers then never sees a phase two ahead)
-    const int64_t x_bytes = (int64_t)nt * 128 * P.xs, c_bytes = kGemmBN * crow;
+    const int64_t x_bytes = (int64_t)nt * 128 * P.xs, c_bytes = kGemmBN * (in.wmode ? crow : crow + 16);
     // codes: 3 chunks (12 stages) for wide token tiles, else up to 6; X slots
     // in the rest (at most 8)
     const int64_t dc_want = in.wmode ? (in.wmode == 1 ? 6 : 4) : nt >= 128 ? 3 : 6;
@@ -792,92 +789,165 @@ gq_status gq_gptq_hessian(const void* d_x, int32_t dtype, int64_t n, int64_t col
     return launch_status();
 }
 
+size_t gq_gptq_batch_workspace_size(const gq_tensor* t, int n) {
+    if (!t || n <= 0) return 0;
+    size_t total = 0;
+    for (int i = 0; i < n; ++i) {
+        if (t[i].rows < 0 || t[i].cols < 0) return 0;
+        total += gptq_layout(nullptr, t[i].rows, t[i].cols).bytes;
+    }
+    return total;
+}
+
+gq_status gq_gptq_quantize_batch(const gq_tensor* t, int n, const double* const* d_H, double percdamp, void* d_ws,
+                                 size_t ws_bytes, int32_t* d_status, cudaStream_t stream) {
+    if (n < 0 || (n > 0 && (!t || !d_H))) return GQ_ERR_INVALID_ARG;
+    if (!(percdamp >= 0.0 && percdamp < 1e6)) return GQ_ERR_INVALID_ARG;
+    if (d_status && !aligned(d_status, 4)) return GQ_ERR_MISALIGNED;
+    size_t need = 0;
+    for (int i = 0; i < n; ++i) {
+        const gq_tensor& T = t[i];
+        gq_status st = check_tensor(T, Op::Export, true);
+        if (st != GQ_OK) return st;
+        if (T.qbits == 16 || T.gran != GQ_PER_ROW || T.col_scale) return GQ_ERR_UNSUPPORTED;
+        if (T.rows == 0 || T.cols == 0) continue;
+        if (!d_H[i]) return GQ_ERR_INVALID_ARG;
+        if (!aligned(d_H[i], 8)) return GQ_ERR_MISALIGNED;
+        if (T.cols > kGptqMaxCols) return GQ_ERR_UNSUPPORTED;
+        need += gptq_layout(nullptr, T.rows, T.cols).bytes;
+    }
+    if (n == 0) return GQ_OK;
+    if (need > 0) {
+        if (!d_ws || ws_bytes < need) return GQ_ERR_WORKSPACE;
+        if (!aligned(d_ws, 256)) return GQ_ERR_MISALIGNED;
+    }
+    if (d_status && cuda_status(cudaMemsetAsync(d_status, 0, sizeof(int32_t) * (size_t)n, stream)) != GQ_OK)
+        return GQ_ERR_CUDA;
+    // the non-empty weights, each with its part of the workspace
+    std::vector<int> idx;
+    std::vector<GptqWs> ws;
+    size_t off = 0;
+    for (int i = 0; i < n; ++i) {
+        if (t[i].rows == 0 || t[i].cols == 0) continue;
+        idx.push_back(i);
+        ws.push_back(gptq_layout(static_cast<unsigned char*>(d_ws) + off, t[i].rows, t[i].cols));
+        off += ws.back().bytes;
+    }
+    if (idx.empty()) return GQ_OK;
+    const int nw = (int)idx.size();
+
+    // 1. clip of every original row (the export's select), into the workspace
+    std::vector<gq_tensor> sel(nw);
+    for (int k = 0; k < nw; ++k) {
+        sel[k] = t[idx[k]];
+        sel[k].dq = nullptr;
+        sel[k].codes = nullptr;
+        sel[k].packed = nullptr;
+        sel[k].scale_f16 = nullptr;
+        sel[k].scale_f32 = nullptr;
+        sel[k].clip = ws[k].clip;
+    }
+    if (nw == n) {
+        // one batched select (status i is tensor i's)
+        gq_status st = quantize_batch(sel.data(), nw, Op::Select, false, nullptr, 0, d_status, stream);
+        if (st != GQ_OK) return st;
+    } else {
+        for (int k = 0; k < nw; ++k) {
+            gq_status st = quantize_batch(&sel[k], 1, Op::Select, false, nullptr, 0,
+                                          d_status ? d_status + idx[k] : nullptr, stream);
+            if (st != GQ_OK) return st;
+        }
+    }
+    for (int k = 0; k < nw; ++k) {
+        const gq_tensor& T = t[idx[k]];
+        if (T.clip && cuda_status(cudaMemcpyAsync(T.clip, ws[k].clip, (size_t)T.rows * 4, cudaMemcpyDeviceToDevice,
+                                                  stream)) != GQ_OK)
+            return GQ_ERR_CUDA;
+    }
+    // 2 - 4 in groups of kGpMaxMats weights
+    const int64_t sms = sm_count();
+    for (int g0 = 0; g0 < nw; g0 += kGpMaxMats) {
+        const int gc = std::min(kGpMaxMats, nw - g0);
+        GpMats M;
+        std::memset(&M, 0, sizeof(M));
+        M.count = gc;
+        int64_t nmax = 0;
+        for (int k = 0; k < gc; ++k) {
+            const int i = idx[g0 + k];
+            GpMat& G = M.m[k];
+            G.H = d_H[i];
+            G.L = ws[g0 + k].L;
+            G.dead = ws[g0 + k].dead;
+            G.st = ws[g0 + k].st;
+            G.n = t[i].cols;
+            nmax = std::max(nmax, G.n);
+        }
+        // 2. dead inputs, damping, reversal
+        gptq_diag_kernel<<<(unsigned)gc, kGpThreads, 0, stream>>>(M, percdamp);
+        const int64_t rev_blocks = std::min<int64_t>(
+            std::max<int64_t>(1, sms * 8 / gc), (nmax * nmax + kGpThreads - 1) / kGpThreads);
+        gptq_reverse_kernel<<<dim3((unsigned)rev_blocks, (unsigned)gc), kGpThreads, 0, stream>>>(M);
+        if (launch_status() != GQ_OK) return GQ_ERR_CUDA;
+        // 3. Cholesky of the reversed, damped Hessians, panel by panel
+        for (int64_t k0 = 0; k0 < nmax; k0 += kGpBlock) {
+            const int64_t below = std::max<int64_t>(0, nmax - k0 - kGpBlock);
+            const unsigned pblocks = (unsigned)std::max<int64_t>(1, (below + 63) / 64);
+            gptq_chol_panel<<<dim3(pblocks, 1, (unsigned)gc), kGpThreads, 0, stream>>>(M, k0);
+            if (below > 0) {
+                const unsigned ut = (unsigned)((below + 63) / 64);
+                gptq_chol_update<<<dim3(ut, ut, (unsigned)gc), kGpThreads, 0, stream>>>(M, k0);
+            }
+            if (launch_status() != GQ_OK) return GQ_ERR_CUDA;
+        }
+        // 4. the recurrence over the rows of every weight of the group
+        GptqParams P;
+        std::memset(&P, 0, sizeof(P));
+        P.ndesc = gc;
+        int64_t blocks = 0;
+        for (int k = 0; k < gc; ++k) {
+            const int i = idx[g0 + k];
+            const gq_tensor& T = t[i];
+            GptqRowDesc& R = P.d[k];
+            R.w = T.w;
+            R.L = ws[g0 + k].L;
+            R.dead = ws[g0 + k].dead;
+            R.st = ws[g0 + k].st;
+            R.clip = ws[g0 + k].clip;
+            R.scale_f16 = T.scale_f16;
+            R.codes = T.codes;
+            R.packed = T.packed;
+            R.dq = T.dq;
+            R.status = d_status ? d_status + i : nullptr;
+            R.rows = T.rows;
+            R.n = T.cols;
+            R.ld = T.ld;
+            R.prb = packed_row_bytes(T.cols, T.qbits);
+            R.start = blocks;
+            R.dtype = T.dtype;
+            R.qbits = T.qbits;
+            blocks += (T.rows + kGpRows - 1) / kGpRows;
+        }
+        P.blocks = blocks;
+        if (P.blocks > INT32_MAX) return GQ_ERR_UNSUPPORTED;
+        const size_t smem = gptq_rows_smem(nmax);
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess) return GQ_ERR_CUDA;
+        if (dev >= 0 && dev < kMaxDevices && g_gptq_smem_set[dev].load() < (int)smem) {
+            if (cuda_status(cudaFuncSetAttribute(gptq_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)smem)) != GQ_OK)
+                return GQ_ERR_CUDA;
+            g_gptq_smem_set[dev].store((int)smem);
+        }
+        gptq_rows_kernel<<<(unsigned)P.blocks, kGpThreads, smem, stream>>>(P);
+        if (launch_status() != GQ_OK) return GQ_ERR_CUDA;
+    }
+    return GQ_OK;
+}
+
 gq_status gq_gptq_quantize(const gq_tensor* t, const double* d_H, double percdamp, void* d_ws, size_t ws_bytes,
                            int32_t* d_status, cudaStream_t stream) {
     if (!t) return GQ_ERR_INVALID_ARG;
-    const gq_tensor& T = *t;
-    gq_status st = check_tensor(T, Op::Export, true);
-    if (st != GQ_OK) return st;
-    if (T.qbits == 16 || T.gran != GQ_PER_ROW || T.col_scale) return GQ_ERR_UNSUPPORTED;
-    if (!(percdamp >= 0.0 && percdamp < 1e6)) return GQ_ERR_INVALID_ARG;
-    if (d_status && !aligned(d_status, 4)) return GQ_ERR_MISALIGNED;
-    if (T.rows == 0 || T.cols == 0) {
-        if (d_status) return cuda_status(cudaMemsetAsync(d_status, 0, sizeof(int32_t), stream));
-        return GQ_OK;
-    }
-    if (!d_H) return GQ_ERR_INVALID_ARG;
-    if (!aligned(d_H, 8)) return GQ_ERR_MISALIGNED;
-    if (T.cols > kGptqMaxCols) return GQ_ERR_UNSUPPORTED;
-    const GptqWs W = gptq_layout(d_ws, T.rows, T.cols);
-    if (!d_ws || ws_bytes < W.bytes) return GQ_ERR_WORKSPACE;
-    if (!aligned(d_ws, 256)) return GQ_ERR_MISALIGNED;
-    const int64_t n = T.cols;
-
-    // 1. clip of every original row (the export's select), into the workspace
-    gq_tensor sel = T;
-    sel.dq = nullptr;
-    sel.codes = nullptr;
-    sel.packed = nullptr;
-    sel.scale_f16 = nullptr;
-    sel.scale_f32 = nullptr;
-    sel.clip = W.clip;
-    st = quantize_batch(&sel, 1, Op::Select, false, nullptr, 0, d_status, stream);
-    if (st != GQ_OK) return st;
-    if (T.clip && cuda_status(cudaMemcpyAsync(T.clip, W.clip, (size_t)T.rows * 4, cudaMemcpyDeviceToDevice,
-                                              stream)) != GQ_OK)
-        return GQ_ERR_CUDA;
-    // 2. dead inputs, damping, reversal
-    gptq_diag_kernel<<<1, kGpThreads, 0, stream>>>(d_H, n, percdamp, W.dead, W.st);
-    const int64_t rev_blocks = std::min<int64_t>((int64_t)sm_count() * 8, (n * n + kGpThreads - 1) / kGpThreads);
-    gptq_reverse_kernel<<<(unsigned)rev_blocks, kGpThreads, 0, stream>>>(d_H, n, W.dead, W.st, W.L);
-    if (launch_status() != GQ_OK) return GQ_ERR_CUDA;
-    // 3. Cholesky of the reversed, damped Hessian
-    for (int64_t k0 = 0; k0 < n; k0 += kGpBlock) {
-        const int64_t nb = std::min<int64_t>(kGpBlock, n - k0);
-        const int64_t below = n - k0 - nb;
-        const unsigned pblocks = (unsigned)std::max<int64_t>(1, (below + 63) / 64);
-        gptq_chol_panel<<<pblocks, kGpThreads, 0, stream>>>(W.L, n, k0, W.st);
-        if (below > 0) {
-            const unsigned ut = (unsigned)((below + 63) / 64);
-            gptq_chol_update<<<dim3(ut, ut), kGpThreads, 0, stream>>>(W.L, n, k0);
-        }
-        if (launch_status() != GQ_OK) return GQ_ERR_CUDA;
-    }
-    // 4. the recurrence over the rows
-    GptqParams P;
-    std::memset(&P, 0, sizeof(P));
-    P.ndesc = 1;
-    GptqRowDesc& R = P.d[0];
-    R.w = T.w;
-    R.L = W.L;
-    R.dead = W.dead;
-    R.st = W.st;
-    R.clip = W.clip;
-    R.scale_f16 = T.scale_f16;
-    R.codes = T.codes;
-    R.packed = T.packed;
-    R.dq = T.dq;
-    R.status = d_status;
-    R.rows = T.rows;
-    R.n = n;
-    R.ld = T.ld;
-    R.prb = packed_row_bytes(n, T.qbits);
-    R.start = 0;
-    R.dtype = T.dtype;
-    R.qbits = T.qbits;
-    P.blocks = (T.rows + kGpRows - 1) / kGpRows;
-    if (P.blocks > INT32_MAX) return GQ_ERR_UNSUPPORTED;
-    const size_t smem = gptq_rows_smem(n);
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return GQ_ERR_CUDA;
-    if (dev >= 0 && dev < kMaxDevices && g_gptq_smem_set[dev].load() < (int)smem) {
-        if (cuda_status(cudaFuncSetAttribute(gptq_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem)) != GQ_OK)
-            return GQ_ERR_CUDA;
-        g_gptq_smem_set[dev].store((int)smem);
-    }
-    gptq_rows_kernel<<<(unsigned)P.blocks, kGpThreads, smem, stream>>>(P);
-    return launch_status();
+    return gq_gptq_quantize_batch(t, 1, &d_H, percdamp, d_ws, ws_bytes, d_status, stream);
 }
 
 gq_status gq_row_clip_select(const gq_tensor* t, int n, void* d_ws, size_t ws_bytes,

@@ -87,6 +87,57 @@ __device__ __forceinline__ void dec_mma(float (&c)[4], uint32_t a0, uint32_t a1,
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Per-row dequant constants as scalars (the same identity as GDeq:
+// q * s = F * S_p - C_p * S_p, one fused multiply-add per code), for
+// scalar fused multiply-adds on the FMA pipe: the decode kernel is bound by
+// the integer pipe, which the register-pair moves of the paired form use.
+struct DecDeq {
+    float s0, c0, s1, c1;        // int6: p = 6, 12; int8 even pair: p = 8, 8
+    float s2, c2, s3, c3;        // int8 odd pair: p = 4, 12
+};
+
+__device__ __forceinline__ DecDeq dec_deq_consts(int qbits, float s) {
+    auto sp = [&](int p) { return __fmul_rn(s, __int_as_float((127 - p) << 23)); };      // s * 2^-p
+    auto cs = [&](int bits, int p) {                                                    // -C_p * S_p
+        return __fmul_rn(-(8388608.0f + (float)(1 << (bits - 1 + p))), sp(p));
+    };
+    DecDeq d;
+    if (qbits == 6) {
+        d.s0 = sp(6); d.c0 = cs(6, 6); d.s1 = sp(12); d.c1 = cs(6, 12);
+        d.s2 = d.c2 = d.s3 = d.c3 = 0.0f;
+    } else {
+        d.s0 = d.s1 = sp(8); d.c0 = d.c1 = cs(8, 8);
+        d.s2 = sp(4); d.c2 = cs(8, 4); d.s3 = sp(12); d.c3 = cs(8, 12);
+    }
+    return d;
+}
+
+// Codes 2i and 2i + 1 of the lane's window w[] (int6: pair i at bit 12 i;
+// int8: bytes 2i, 2i + 1) as one bf16x2 word of W_hat; the fields are those
+// of g_pair.
+template <int QBITS>
+__device__ __forceinline__ uint32_t dec_pair(const uint32_t (&w)[16], int i, const DecDeq& d) {
+    if constexpr (QBITS == 6) {
+        uint32_t v;
+        if (i == 0) {
+            v = w[0] << 6;
+        } else {
+            const int sh = 12 * i - 6;
+            v = __funnelshift_r(w[sh >> 5], w[(sh >> 5) + 1], sh & 31);
+        }
+        return g_bf16x2(__fmaf_rn(g_field(v, 0xFC0u, 0x4B000800u), d.s0, d.c0),
+                        __fmaf_rn(g_field(v, 0x3F000u, 0x4B020000u), d.s1, d.c1));
+    } else {
+        const uint32_t wd = w[i >> 1];
+        if ((i & 1) == 0)
+            return g_bf16x2(__fmaf_rn(g_field(wd << 8, 0xFF00u, 0x4B008000u), d.s0, d.c0),
+                            __fmaf_rn(g_field(wd, 0xFF00u, 0x4B008000u), d.s1, d.c1));
+        const uint32_t v = wd >> 12;
+        return g_bf16x2(__fmaf_rn(g_field(v, 0xFF0u, 0x4B000800u), d.s2, d.c2),
+                        __fmaf_rn(g_field(v, 0xFF000u, 0x4B080000u), d.s3, d.c3));
+    }
+}
+
 // Byte offset of 16-byte chunk c (0 .. 63) of X slice row m: chunk c sits
 // at position c ^ ((c >> 3) & 7), so that the four lanes of a quad, which
 // read chunks 32 ss + 8 t + i at the same time, hit different banks (and
@@ -157,7 +208,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) gemm_decode_kernel(const __gri
     // ---- compute side
     int64_t cp_nb = u0 / P.kunits, cp_kb = u0 - cp_nb * P.kunits;
     float acc[kDecNG][4];
-    GDeq deq[kDecNG];
+    DecDeq deq[kDecNG];
     int64_t cur_nb = -1;
     auto flush = [&]() {
         // lane holds Y[g][n], Y[g][n + 1], Y[g + 8][n], Y[g + 8][n + 1], n = row block + 8 j + 2 t
@@ -205,7 +256,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) gemm_decode_kernel(const __gri
                     acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
                     const int64_t n = cp_nb * kDecRows + row_lane + 8 * j;
                     const float srow = n < P.N ? __half2float(__ushort_as_half(P.scale[n])) : 0.0f;
-                    deq[j] = g_deq_consts(QBITS, srow);
+                    deq[j] = dec_deq_consts(QBITS, srow);
                 }
             }
         }
@@ -234,25 +285,29 @@ __global__ void __launch_bounds__(kDecThreads, 1) gemm_decode_kernel(const __gri
 #pragma unroll
                 for (int w = 4 * LC; w < 16; ++w) cw[j][w] = 0u;
             }
+            // X rows g and g + 8 of this super-stage: chunk 32 ss + 8 t + q sits at
+            // 32 ss + 8 t + (q ^ r), r = (4 ss + t) & 7 (dec_x_off)
+            const uint32_t xg = xb + (uint32_t)(g * kDecPitch) * 2u + 16u * (uint32_t)(32 * ss + 8 * t);
+            const uint32_t r = (uint32_t)((4 * ss + t) & 7);
 #pragma unroll
             for (int s = 0; s < 4; ++s) {
-                // X rows g and g + 8, physical pairs 32 t + 8 s .. + 7: chunks 32 ss + 8 t + 2 s, + 1
+                // physical pairs 32 t + 8 s .. + 7: chunks q = 2 s, 2 s + 1 of the lane's eight
                 uint32_t xa[8], xc[8];
-                const int c0 = 32 * ss + 8 * t + 2 * s;
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
+                    const uint32_t a = xg + 16u * (((uint32_t)(2 * s + h)) ^ r);
                     asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                                  : "=r"(xa[4 * h]), "=r"(xa[4 * h + 1]), "=r"(xa[4 * h + 2]), "=r"(xa[4 * h + 3])
-                                 : "r"(xb + dec_x_off(g, c0 + h)));
+                                 : "r"(a));
                     asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                                  : "=r"(xc[4 * h]), "=r"(xc[4 * h + 1]), "=r"(xc[4 * h + 2]), "=r"(xc[4 * h + 3])
-                                 : "r"(xb + dec_x_off(g + 8, c0 + h)));
+                                 : "r"(a + (uint32_t)(8 * kDecPitch) * 2u));
                 }
 #pragma unroll
                 for (int j = 0; j < kDecNG; ++j) {
                     uint32_t wp[8];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) wp[i] = g_pair<QBITS>(cw[j], 8 * s + i, deq[j]);
+                    for (int i = 0; i < 8; ++i) wp[i] = dec_pair<QBITS>(cw[j], 8 * s + i, deq[j]);
 #pragma unroll
                     for (int b = 0; b < 4; ++b)
                         dec_mma(acc[j], xa[2 * b], xc[2 * b], xa[2 * b + 1], xc[2 * b + 1], wp[2 * b], wp[2 * b + 1]);

@@ -113,11 +113,31 @@ struct GpState {
     int32_t bad;         // non-finite or non-positive pivot met
 };
 
-// One block: dead inputs (H[j, j] == 0 -> flagged, treated as 1) and
-// lambda = percdamp * mean(diag H) over the fixed diagonal.
-__global__ void __launch_bounds__(kGpThreads) gptq_diag_kernel(const double* __restrict__ H, int64_t n,
-                                                               double percdamp, uint8_t* __restrict__ dead,
-                                                               GpState* st) {
+// The per-weight matrices of a batch: the kernels below take their matrix
+// from a grid index, so that the independent chains of several weights run
+// in the same launches.
+struct GpMat {
+    const double* H;     // [n, n] Hessian (input)
+    double* L;           // [n, n] reversed, damped Hessian, then its lower factor
+    uint8_t* dead;       // [n]
+    GpState* st;
+    int64_t n;
+};
+constexpr int kGpMaxMats = 64;
+struct GpMats {
+    int32_t count;
+    int32_t pad;
+    GpMat m[kGpMaxMats];
+};
+
+// One block per matrix: dead inputs (H[j, j] == 0 -> flagged, treated as 1)
+// and lambda = percdamp * mean(diag H) over the fixed diagonal.
+__global__ void __launch_bounds__(kGpThreads) gptq_diag_kernel(const __grid_constant__ GpMats M, double percdamp) {
+    const GpMat& G = M.m[blockIdx.x];
+    const double* __restrict__ H = G.H;
+    const int64_t n = G.n;
+    uint8_t* __restrict__ dead = G.dead;
+    GpState* st = G.st;
     __shared__ double part[kGpThreads];
     __shared__ int cnt[kGpThreads];
     double sum = 0.0;
@@ -149,11 +169,14 @@ __global__ void __launch_bounds__(kGpThreads) gptq_diag_kernel(const double* __r
 // Hr[a, b] = Hd[n-1-a, n-1-b] for b <= a, Hd = H with dead diagonals set to 1
 // and lambda added to the diagonal (a dead input also drops out of the
 // off-diagonal coupling: its weights are zeroed, so its row of H is unused).
-__global__ void __launch_bounds__(kGpThreads) gptq_reverse_kernel(const double* __restrict__ H, int64_t n,
-                                                                  const uint8_t* __restrict__ dead,
-                                                                  const GpState* __restrict__ st,
-                                                                  double* __restrict__ Hr) {
-    const double lam = st->lambda;
+// (matrix blockIdx.y of the batch; the x blocks stride over its entries)
+__global__ void __launch_bounds__(kGpThreads) gptq_reverse_kernel(const __grid_constant__ GpMats M) {
+    const GpMat& G = M.m[blockIdx.y];
+    const double* __restrict__ H = G.H;
+    const int64_t n = G.n;
+    const uint8_t* __restrict__ dead = G.dead;
+    double* __restrict__ Hr = G.L;
+    const double lam = G.st->lambda;
     const int64_t total = n * n;
     for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
         const int64_t a = e / n, b = e % n;
@@ -172,8 +195,15 @@ __global__ void __launch_bounds__(kGpThreads) gptq_reverse_kernel(const double* 
 // trailing updates of earlier panels are already applied), block 0 writes it
 // back, and each block solves 64 rows below it: L[i, k0 + c] =
 // (A[i, k0 + c] - sum_{d < c} L[i, k0 + d] L[k0 + c, k0 + d]) / L[k0 + c, k0 + c].
-__global__ void __launch_bounds__(kGpThreads) gptq_chol_panel(double* __restrict__ A, int64_t n, int64_t k0,
-                                                              GpState* st) {
+// (matrix blockIdx.z of the batch; a matrix whose order is at most k0 has no
+// panel here, and x blocks past its own row count do nothing)
+__global__ void __launch_bounds__(kGpThreads) gptq_chol_panel(const __grid_constant__ GpMats M, int64_t k0) {
+    const GpMat& G = M.m[blockIdx.z];
+    const int64_t n = G.n;
+    if (k0 >= n) return;
+    if ((int64_t)blockIdx.x * 64 >= max((int64_t)1, n - k0 - kGpBlock)) return;
+    double* __restrict__ A = G.L;
+    GpState* st = G.st;
     __shared__ double D[kGpBlock][kGpBlock + 1];
     const int nb = (int)min((int64_t)kGpBlock, n - k0);
     const int t = threadIdx.x;
@@ -225,11 +255,16 @@ __global__ void __launch_bounds__(kGpThreads) gptq_chol_panel(double* __restrict
 // Trailing update after panel k0: A[i, j] -= sum_c L[i, k0 + c] L[j, k0 + c]
 // for k0 + nb <= j <= i, on 64 x 64 tiles of the lower triangle; the panel
 // columns are staged 32 at a time.
-__global__ void __launch_bounds__(kGpThreads) gptq_chol_update(double* __restrict__ A, int64_t n, int64_t k0) {
+// (matrix blockIdx.z of the batch; tiles past its own trailing block do nothing)
+__global__ void __launch_bounds__(kGpThreads) gptq_chol_update(const __grid_constant__ GpMats M, int64_t k0) {
+    const GpMat& G = M.m[blockIdx.z];
+    const int64_t n = G.n;
     const int ti = blockIdx.y, tj = blockIdx.x;
-    if (tj > ti) return;
-    const int nb = (int)min((int64_t)kGpBlock, n - k0);
+    if (tj > ti || k0 + kGpBlock >= n) return;
+    double* __restrict__ A = G.L;
+    const int nb = kGpBlock;
     const int64_t base = k0 + nb;
+    if (base + (int64_t)ti * 64 >= n) return;
     const int64_t i0 = base + (int64_t)ti * 64, j0 = base + (int64_t)tj * 64;
     constexpr int kCh = 32;
     __shared__ double Pi[64][kCh + 1];
@@ -288,7 +323,7 @@ struct GptqRowDesc {
     int32_t dtype, qbits;
 };
 
-constexpr int kGpMaxDesc = 32;
+constexpr int kGpMaxDesc = kGpMaxMats;
 
 struct GptqParams {
     int32_t ndesc;

@@ -42,7 +42,7 @@ EXPORTED = ("gq_row_clip_select", "gq_fakequant_fwd", "gq_fakequant_average", "g
             "gq_export_pack_noalloc", "gq_dequant", "gq_gemm_dequant", "gq_workspace_size", "gq_packed_row_bytes", "gq_k_from_p",
             "gq_plan_kind", "gq_status_string", "gq_last_cuda_error", "gq_last_cuda_error_string",
             "gq_test_arm_wait_expiry", "gq_gptq_quantize", "gq_gptq_hessian", "gq_gptq_workspace_size",
-            "gq_gemm_fakequant")
+            "gq_gemm_fakequant", "gq_gptq_quantize_batch", "gq_gptq_batch_workspace_size")
 
 
 class GQError(RuntimeError):
@@ -90,6 +90,10 @@ def _load() -> C.CDLL:
         getattr(L, f).restype = i32
     L.gq_gptq_quantize.argtypes = [T, vp, f64, vp, sz, vp, vp]
     L.gq_gptq_quantize.restype = i32
+    L.gq_gptq_quantize_batch.argtypes = [T, i32, C.POINTER(vp), f64, vp, sz, vp, vp]
+    L.gq_gptq_quantize_batch.restype = i32
+    L.gq_gptq_batch_workspace_size.argtypes = [T, i32]
+    L.gq_gptq_batch_workspace_size.restype = sz
     L.gq_gptq_hessian.argtypes = [vp, i32, i64, i64, i64, vp, i32, vp]
     L.gq_gptq_hessian.restype = i32
     L.gq_gptq_workspace_size.argtypes = [i64, i64]
@@ -451,6 +455,38 @@ def gptq_quantize(req: Request, H: torch.Tensor, percdamp: float = 0.01, stream=
     if check_status:
         o.status = int(st[0].item())
     return o
+
+
+def gptq_quantize_batch(reqs, Hs, percdamp: float = 0.01, stream=None,
+                        check_status: bool = True) -> list:
+    """GPTQ-lite of several weights in one call (gq_gptq_quantize_batch): the
+    outputs of gptq_quantize for each (request, Hessian) pair, bitwise."""
+    if len(reqs) != len(Hs):
+        raise ValueError("one Hessian per request")
+    rs = []
+    for req in reqs:
+        if req.per_tensor or req.qbits not in (6, 8) or req.col_scale is not None:
+            raise ValueError("GPTQ-lite takes per-row int6 / int8 requests without column scales")
+        rs.append(Request(**{**req.__dict__, "want_packed": True, "want_scale_f16": True, "want_scale_f32": False}))
+    descs, outs = _prepare(rs, True)
+    for d, H in zip(descs, Hs):
+        if H.dtype != torch.float64 or not H.is_contiguous() or H.shape != (d.cols, d.cols):
+            raise ValueError("each H must be a contiguous fp64 [cols, cols] tensor")
+    if not descs:
+        return outs
+    dev = reqs[0].w.device
+    arr = _arr(descs)
+    nbytes = LIB.gq_gptq_batch_workspace_size(arr, len(descs))
+    ws = _SCRATCH.workspace(dev, nbytes)
+    st = _SCRATCH.status(dev, len(descs))
+    hp = (C.c_void_p * len(descs))(*[H.data_ptr() for H in Hs])
+    _check(LIB.gq_gptq_quantize_batch(arr, len(descs), hp, float(percdamp), ws.data_ptr(), ws.numel(),
+                                      st.data_ptr(), _stream(stream)), "gq_gptq_quantize_batch")
+    if check_status:
+        sv = st[:len(descs)].cpu().tolist()
+        for o, v in zip(outs, sv):
+            o.status = int(v)
+    return outs
 
 
 def gemm_fakequant(x: torch.Tensor, w: torch.Tensor, clip: torch.Tensor, qbits: int = 6,

@@ -161,3 +161,72 @@ def test_gptq_argument_errors(gq):
     d.cols = 6000
     d.ld = 6000
     assert gq.LIB.gq_gptq_quantize(C.byref(d), H.data_ptr(), 0.01, None, 0, None, None) == 2   # too wide
+
+
+def test_gptq_batch_equals_single_calls(gq):
+    """gq_gptq_quantize_batch over weights of different shapes, dtypes and
+    bit widths gives, bitwise, the outputs of one gq_gptq_quantize per
+    weight (whose parity with the oracle the tests above check)."""
+    rng = np.random.default_rng(44)
+    shapes = [(96, 200, "f32", 6, 1.0), (130, 517, "bf16", 6, 0.999), (40, 1584, "f32", 6, 0.9999),
+              (33, 64, "f32", 8, 1.0), (256, 528, "bf16", 6, 1.0)]
+    reqs, Hs = [], []
+    for rows, cols, dt, qbits, p in shapes:
+        w = synth.random_matrix(rng, rows, cols, "t3")
+        if dt == "bf16":
+            w = synth.to_bf16_bits(w).reshape(rows, cols)
+        reqs.append(gq.Request(_dev(w), qbits, p, want_dq=True, want_codes=True, want_clip=True))
+        Hs.append(gq.gptq_hessian(_dev(synth.gptq_calibration(rng, 300, cols))))
+    outs = gq.gptq_quantize_batch(reqs, Hs)
+    for r, H, o in zip(reqs, Hs, outs):
+        one = gq.gptq_quantize(gq.Request(r.w, r.qbits, r.p, want_dq=True, want_codes=True, want_clip=True), H)
+        torch.cuda.synchronize()
+        assert o.status == 0 and one.status == 0
+        assert torch.equal(o.codes, one.codes) and torch.equal(o.packed, one.packed)
+        assert torch.equal(o.scale_f16.view(torch.int16), one.scale_f16.view(torch.int16))
+        assert torch.equal(o.dq.view(torch.int16) if o.dq.dtype == torch.bfloat16 else o.dq.view(torch.int32),
+                           one.dq.view(torch.int16) if one.dq.dtype == torch.bfloat16 else one.dq.view(torch.int32))
+        assert torch.equal(o.clip.view(torch.int32), one.clip.view(torch.int32))
+
+
+def test_gptq_batch_unified11_model(gq):
+    """All 44 weights of the 11-layer d528 model in one batched call: each
+    equal to its single call, and the first layer's four against the oracle."""
+    ws = synth.draw_unified11()
+    specs = synth.unified11_train().specs
+    rng = np.random.default_rng(22)
+    xs = [synth.gptq_calibration(rng, 512, s.shape[1]) for s in specs]
+    reqs = [gq.Request(_dev(ws[s.name]), 6, 1.0, want_dq=True, want_codes=True) for s in specs]
+    Hs = [gq.gptq_hessian(_dev(x)) for x in xs]
+    outs = gq.gptq_quantize_batch(reqs, Hs)
+    for i, (s, r, H, o) in enumerate(zip(specs, reqs, Hs, outs)):
+        assert o.status == 0, s.name
+        if i % 7 == 0:
+            one = gq.gptq_quantize(gq.Request(r.w, 6, 1.0, want_dq=True, want_codes=True), H)
+            torch.cuda.synchronize()
+            assert torch.equal(o.codes, one.codes) and torch.equal(o.packed, one.packed), s.name
+    for i in range(4):
+        ref = G.gptq(ws[specs[i].name], G.hessian(xs[i]), 6, 1.0)
+        codes = _host(outs[i].codes)
+        bad = np.nonzero((codes != ref.codes).any(axis=1))[0]
+        for r in bad:
+            j = int(np.nonzero(codes[r] != ref.codes[r])[0][0])
+            t = ref.quotient[r, j]
+            assert abs(abs(t - np.floor(t)) - 0.5) < 1e-6, (specs[i].name, r, j, t)
+        assert len(bad) <= max(1, codes.shape[0] // 100)
+
+
+def test_gptq_batch_argument_errors(gq):
+    import ctypes as C
+    W = torch.zeros(8, 16, device="cuda")
+    H = torch.eye(16, dtype=torch.float64, device="cuda")
+    d = gq.GQTensor(w=W.data_ptr(), dtype=0, qbits=6, gran=0, reserved=0, rows=8, cols=16, ld=16, p=1.0,
+                    dq=0, codes=0, packed=W.data_ptr(), scale_f16=W.data_ptr(), scale_f32=0, clip=0)
+    arr = gq._arr([d, d])
+    hp = (C.c_void_p * 2)(H.data_ptr(), H.data_ptr())
+    L = gq.LIB
+    assert L.gq_gptq_batch_workspace_size(arr, 2) == 2 * L.gq_gptq_workspace_size(8, 16)
+    assert L.gq_gptq_quantize_batch(arr, 2, hp, 0.01, None, 0, None, None) == 4        # no workspace
+    assert L.gq_gptq_quantize_batch(arr, 2, None, 0.01, None, 0, None, None) == 1      # no Hessians
+    assert L.gq_gptq_quantize_batch(arr, 2, hp, -1.0, None, 0, None, None) == 1        # bad percdamp
+    assert L.gq_gptq_quantize_batch(arr, 0, hp, 0.01, None, 0, None, None) == 0        # nothing to do
