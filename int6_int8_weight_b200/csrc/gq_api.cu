@@ -549,7 +549,8 @@ GptqWs gptq_layout(void* base, int64_t rows, int64_t cols) {
     return w;
 }
 
-std::atomic<int> g_gptq_smem_set[kMaxDevices];
+std::atomic<int> g_gptq_smem_set[2][kMaxDevices];
+constexpr int kGptqSmemLimit = 232448 - 1024;     // dynamic shared memory of a block (static arrays aside)
 
 struct GemmIn {
     const void* x;
@@ -703,13 +704,10 @@ gq_status gemm_launch(const GemmIn& in) {
                 return GQ_ERR_UNSUPPORTED;
         }
     } else if (tma_codes) {
-        // packed rows as {16 bytes, prb / 16 chunks, N rows}; a copy takes one
-        // chunk more than the row's stages hold, which pads the rows in shared
-        // memory to an odd number of chunks (no bank conflicts)
-        const cuuint64_t wdim[3] = {16, (cuuint64_t)(prb / 16), (cuuint64_t)N};
-        const cuuint64_t wstride[2] = {16, (cuuint64_t)prb};
-        const cuuint32_t wbox[3] = {16, (cuuint32_t)(crow / 16 + 1), (cuuint32_t)kGemmBN};
-        if (enc(&P.tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(d_packed), wdim, wstride, wbox,
+        const cuuint64_t wdim[2] = {(cuuint64_t)prb, (cuuint64_t)N};
+        const cuuint64_t wstride[1] = {(cuuint64_t)prb};
+        const cuuint32_t wbox[2] = {(cuuint32_t)crow, (cuuint32_t)kGemmBN};
+        if (enc(&P.tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(d_packed), wdim, wstride, wbox,
                 estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return GQ_ERR_UNSUPPORTED;
@@ -741,7 +739,7 @@ gq_status gemm_launch(const GemmIn& in) {
     // is left, W_hat in the TMEM columns after the accumulators; the commit
     // ring is a multiple of the W_hat depth and at least the X depth (a
     // waiter on any of these barriers then never sees a phase two ahead)
-    const int64_t x_bytes = (int64_t)nt * 128 * P.xs, c_bytes = kGemmBN * (in.wmode ? crow : crow + 16);
+    const int64_t x_bytes = (int64_t)nt * 128 * P.xs, c_bytes = kGemmBN * crow;
     // codes: 3 chunks (12 stages) for wide token tiles, else up to 6; X slots
     // in the rest (at most 8)
     const int64_t dc_want = in.wmode ? (in.wmode == 1 ? 6 : 4) : nt >= 128 ? 3 : 6;
@@ -899,7 +897,9 @@ gq_status gq_gptq_quantize_batch(const gq_tensor* t, int n, const double* const*
             }
             if (launch_status() != GQ_OK) return GQ_ERR_CUDA;
         }
-        // 4. the recurrence over the rows of every weight of the group
+        // 4. the recurrence over the rows of every weight of the group, 8 rows
+        // per block when their residuals fit in shared memory, else 4
+        const int rpb = gptq_rows_smem(nmax, 8) <= (size_t)kGptqSmemLimit ? 8 : 4;
         GptqParams P;
         std::memset(&P, 0, sizeof(P));
         P.ndesc = gc;
@@ -925,20 +925,22 @@ gq_status gq_gptq_quantize_batch(const gq_tensor* t, int n, const double* const*
             R.start = blocks;
             R.dtype = T.dtype;
             R.qbits = T.qbits;
-            blocks += (T.rows + kGpRows - 1) / kGpRows;
+            blocks += (T.rows + rpb - 1) / rpb;
         }
         P.blocks = blocks;
         if (P.blocks > INT32_MAX) return GQ_ERR_UNSUPPORTED;
-        const size_t smem = gptq_rows_smem(nmax);
+        const size_t smem = gptq_rows_smem(nmax, rpb);
         int dev = 0;
         if (cudaGetDevice(&dev) != cudaSuccess) return GQ_ERR_CUDA;
-        if (dev >= 0 && dev < kMaxDevices && g_gptq_smem_set[dev].load() < (int)smem) {
-            if (cuda_status(cudaFuncSetAttribute(gptq_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)smem)) != GQ_OK)
+        const int ri = rpb == 8 ? 1 : 0;
+        if (dev >= 0 && dev < kMaxDevices && g_gptq_smem_set[ri][dev].load() < (int)smem) {
+            if (cuda_status(cudaFuncSetAttribute(ri ? gptq_rows_kernel<8> : gptq_rows_kernel<4>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != GQ_OK)
                 return GQ_ERR_CUDA;
-            g_gptq_smem_set[dev].store((int)smem);
+            g_gptq_smem_set[ri][dev].store((int)smem);
         }
-        gptq_rows_kernel<<<(unsigned)P.blocks, kGpThreads, smem, stream>>>(P);
+        if (ri) gptq_rows_kernel<8><<<(unsigned)P.blocks, kGpThreads, smem, stream>>>(P);
+        else gptq_rows_kernel<4><<<(unsigned)P.blocks, kGpThreads, smem, stream>>>(P);
         if (launch_status() != GQ_OK) return GQ_ERR_CUDA;
     }
     return GQ_OK;

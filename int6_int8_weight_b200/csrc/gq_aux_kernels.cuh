@@ -224,6 +224,10 @@ ste_kernel(const void* __restrict__ g_out, void* __restrict__ g_w, int dtype, in
 // `words` (int6: cols a multiple of 16 and 4-byte aligned rows; int8: cols a
 // multiple of 4 and aligned rows) lanes read aligned 32-bit words and the
 // 24-bit int6 groups are reassembled with two shuffles; otherwise bytes.
+// The code words of kDqUnroll steps are loaded before any of them is used,
+// so that a warp keeps that many loads in flight instead of one.
+constexpr int kDqUnroll = 4;
+
 __global__ void __launch_bounds__(kBlockThreads)
 dequant_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ sf16, int qbits,
                int per_tensor, int64_t rows, int64_t cols, int64_t prb, void* __restrict__ out,
@@ -241,63 +245,75 @@ dequant_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ 
         const uint16_t hb = sf16[per_tensor ? 0 : r];
         const float s = __half2float(*reinterpret_cast<const __half*>(&hb));
         const uint8_t* prow = packed + r * prb;
-        for (int jb = 0; jb < nq; jb += 32) {
-            const int j = jb + lane;
-            const bool valid = j < nq;
-            const int e0 = 4 * j;
-            int q[4];
-            if (qbits == 6) {
-                uint32_t v;
-                if (words) {
-                    uint32_t word = 0u;
-                    if (valid && sub < 3) word = reinterpret_cast<const uint32_t*>(prow + 3 * (j - sub))[sub];
-                    const uint32_t lo = __shfl_sync(0xFFFFFFFFu, word, base + a);
-                    const uint32_t hi = __shfl_sync(0xFFFFFFFFu, word, base + a + 1);
-                    v = __funnelshift_r(lo, hi, shift);
-                } else {
-                    v = 0u;
-                    if (valid)
-                        v = (uint32_t)prow[3 * j] | ((uint32_t)prow[3 * j + 1] << 8) |
-                            ((uint32_t)prow[3 * j + 2] << 16);
-                }
+        for (int jb0 = 0; jb0 < nq; jb0 += 32 * kDqUnroll) {
+            // the code words (or bytes) of kDqUnroll steps, loaded first
+            uint32_t raw[kDqUnroll];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) q[i] = ((int32_t)(v << (26 - 6 * i))) >> 26;   // sign-extend 6 bits
-            } else {
+            for (int u = 0; u < kDqUnroll; ++u) {
+                const int j = jb0 + 32 * u + lane;
+                const bool valid = j < nq;
+                const int e0 = 4 * j;
                 uint32_t v = 0u;
-                if (valid) {
+                if (qbits == 6) {
                     if (words) {
-                        v = *reinterpret_cast<const uint32_t*>(prow + e0);
+                        if (valid && sub < 3) v = __ldg(reinterpret_cast<const uint32_t*>(prow + 3 * (j - sub)) + sub);
+                    } else if (valid) {
+                        v = (uint32_t)prow[3 * j] | ((uint32_t)prow[3 * j + 1] << 8) | ((uint32_t)prow[3 * j + 2] << 16);
+                    }
+                } else if (valid) {
+                    if (words) {
+                        v = __ldg(reinterpret_cast<const uint32_t*>(prow + e0));
                     } else {
 #pragma unroll
                         for (int i = 0; i < 4; ++i)
                             if (e0 + i < cols) v |= (uint32_t)prow[e0 + i] << (8 * i);
                     }
                 }
-#pragma unroll
-                for (int i = 0; i < 4; ++i) q[i] = ((int32_t)(v << (24 - 8 * i))) >> 24;
+                raw[u] = v;
             }
-            if (!valid) continue;
-            float d[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) d[i] = __fmul_rn((float)q[i], s);
-            const bool full = e0 + 3 < cols;
-            if (out_dtype == kF32) {
-                float* o = reinterpret_cast<float*>(out) + r * cols;
-                if (vec_out && full) {
-                    *reinterpret_cast<float4*>(o + e0) = make_float4(d[0], d[1], d[2], d[3]);
+            for (int u = 0; u < kDqUnroll; ++u) {
+                const int j = jb0 + 32 * u + lane;
+                const bool valid = j < nq;
+                const int e0 = 4 * j;
+                int q[4];
+                if (qbits == 6) {
+                    uint32_t v = raw[u];
+                    if (words) {
+                        // every lane takes part in the shuffles, valid or not
+                        const uint32_t lo = __shfl_sync(0xFFFFFFFFu, raw[u], base + a);
+                        const uint32_t hi = __shfl_sync(0xFFFFFFFFu, raw[u], base + a + 1);
+                        v = __funnelshift_r(lo, hi, shift);
+                    }
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) q[i] = ((int32_t)(v << (26 - 6 * i))) >> 26;   // sign-extend 6 bits
                 } else {
-                    for (int i = 0; i < 4; ++i)
-                        if (e0 + i < cols) o[e0 + i] = d[i];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) q[i] = ((int32_t)(raw[u] << (24 - 8 * i))) >> 24;
                 }
-            } else {
-                uint16_t* o = reinterpret_cast<uint16_t*>(out) + r * cols;
-                if (vec_out && full) {
-                    *reinterpret_cast<uint2*>(o + e0) =
-                        make_uint2((uint32_t)float_to_bf16_bits(d[0]) | ((uint32_t)float_to_bf16_bits(d[1]) << 16),
-                                   (uint32_t)float_to_bf16_bits(d[2]) | ((uint32_t)float_to_bf16_bits(d[3]) << 16));
+                if (!valid) continue;
+                float d[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) d[i] = __fmul_rn((float)q[i], s);
+                const bool full = e0 + 3 < cols;
+                if (out_dtype == kF32) {
+                    float* o = reinterpret_cast<float*>(out) + r * cols;
+                    if (vec_out && full) {
+                        *reinterpret_cast<float4*>(o + e0) = make_float4(d[0], d[1], d[2], d[3]);
+                    } else {
+                        for (int i = 0; i < 4; ++i)
+                            if (e0 + i < cols) o[e0 + i] = d[i];
+                    }
                 } else {
-                    for (int i = 0; i < 4; ++i)
-                        if (e0 + i < cols) o[e0 + i] = float_to_bf16_bits(d[i]);
+                    uint16_t* o = reinterpret_cast<uint16_t*>(out) + r * cols;
+                    if (vec_out && full) {
+                        *reinterpret_cast<uint2*>(o + e0) =
+                            make_uint2((uint32_t)float_to_bf16_bits(d[0]) | ((uint32_t)float_to_bf16_bits(d[1]) << 16),
+                                       (uint32_t)float_to_bf16_bits(d[2]) | ((uint32_t)float_to_bf16_bits(d[3]) << 16));
+                    } else {
+                        for (int i = 0; i < 4; ++i)
+                            if (e0 + i < cols) o[e0 + i] = float_to_bf16_bits(d[i]);
+                    }
                 }
             }
         }

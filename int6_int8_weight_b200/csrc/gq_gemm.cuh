@@ -76,7 +76,7 @@ constexpr unsigned long long kGemmWaitNs = 4000000000ull;
 
 struct GemmParams {
     CUtensorMap tmap_x;          // X: 3-D {64, M, K / 64} box {64, nt, CS}, or 2-D [M, K] box {64, nt}; SWIZZLE_128B
-    CUtensorMap tmap_w;          // codes: 3-D {16, prb / 16, N} bytes, box {16, CS stages' chunks + 1, 128} (TMA mode)
+    CUtensorMap tmap_w;          // codes [N, prb] bytes, box (CS stages' bytes) x 128, no swizzle (TMA mode)
     const uint8_t* codes;        // packed codes (copy mode)
     const uint16_t* scale;       // [N] binary16 row scales (codes)
     const float* clip;           // [N] row clips (weight modes)
@@ -610,12 +610,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_dequant_kernel(const __g
     // row; fp32: two 128-byte halves, 16 KB apart)
     const uint32_t cb = P.wmode == 1 ? 128u : P.wmode == 2 ? 256u : P.qbits == 6 ? 48u : 64u;
     const uint32_t crow = cb * (uint32_t)CS;               // bytes of a row's chunk
-    // row pitch in a code slot: packed rows get 16 bytes of padding (the code
-    // copy carries one more 16-byte chunk per row), so that the 8 rows a
-    // quarter warp reads at once (pitch 208 / 272 bytes, 13 / 17 chunks)
-    // fall on different banks; the weight modes keep their swizzled rows
-    const uint32_t cpitch = WM == 0 ? crow + 16u : crow;
-    const uint32_t c_bytes = (uint32_t)kGemmBN * cpitch;   // a code chunk slot
+    const uint32_t c_bytes = (uint32_t)kGemmBN * crow;     // a code chunk slot
     // [X ring][code ring][barriers]
     const uint32_t cs0 = base + (uint32_t)DX * x_bytes;
     const uint32_t bars = base + (uint32_t)(kGemmSmemBytes - 1024 - kGemmBarBytes);
@@ -712,10 +707,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_dequant_kernel(const __g
                 }
             } else if (!P.code_copy) {
                 if (lane == 0) {
-                    // 3-D view {16 bytes, chunks of 16, rows}: crow / 16 + 1 chunks per row;
-                    // out-of-range rows / bytes are zero-filled
-                    g_arrive_tx(full_c(rc.s), c_bytes);
-                    g_tma_load_3d(c_tile(rc.s), &P.tmap_w, 0, it.c * (int)(crow / 16u), n0, full_c(rc.s));
+                    g_arrive_tx(full_c(rc.s), c_bytes);    // out-of-range rows / bytes are zero-filled
+                    g_tma_load_2d(c_tile(rc.s), &P.tmap_w, it.c * (int)crow, n0, full_c(rc.s));
                 }
             } else {
                 // 4-byte copies of every row's chunk bytes; past the row end
@@ -728,7 +721,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_dequant_kernel(const __g
                     const int64_t off = off0 + 4 * wi;
                     const bool in = n < P.N && off + 4 <= P.prb;
                     const uint8_t* src = in ? P.codes + n * P.prb + off : P.codes;
-                    g_cp_async4(c_tile(rc.s) + r * cpitch + 4u * wi, src, in ? 4u : 0u);
+                    g_cp_async4(c_tile(rc.s) + r * crow + 4u * wi, src, in ? 4u : 0u);
                 }
                 g_cp_async_arrive(full_c(rc.s));
             }
@@ -931,7 +924,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_dequant_kernel(const __g
                 break;
             }
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            const uint32_t codes = c_tile(rc.s) + (uint32_t)r * cpitch + (uint32_t)k * cb;
+            const uint32_t codes = c_tile(rc.s) + (uint32_t)r * crow + (uint32_t)k * cb;
             const uint32_t taddr = lane_addr + 32u * (uint32_t)(rw.s * CS + k);
             if constexpr (WM != 0) {
                 if (P.wmode == 1) g_fakequant_stage<kBF16>(c_tile(rc.s), r, taddr, fq);
