@@ -291,10 +291,10 @@ class Workload:
         want = []
         for dt in ("f32", "bf16"):
             for i, (r, c) in enumerate(synth.BANDWIDTH_SHAPES):
-                r = r // shrink
+                # calls are named by the full-size shape, also when shrunken
                 names = [f"{dt} {r}x{c} int{q}" for q in (6, 8)]
                 if only is None or any(only in nm for nm in names):
-                    want.append((dt, i, r, c))
+                    want.append((dt, i, r // shrink, c))
         mats32 = {}
         for dt, i, r, c in want:
             if i not in mats32:

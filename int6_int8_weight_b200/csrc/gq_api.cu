@@ -549,8 +549,7 @@ GptqWs gptq_layout(void* base, int64_t rows, int64_t cols) {
     return w;
 }
 
-std::atomic<int> g_gptq_smem_set[2][kMaxDevices];
-constexpr int kGptqSmemLimit = 232448 - 1024;     // dynamic shared memory of a block (static arrays aside)
+std::atomic<int> g_gptq_smem_set[kMaxDevices];
 
 struct GemmIn {
     const void* x;
@@ -897,51 +896,62 @@ gq_status gq_gptq_quantize_batch(const gq_tensor* t, int n, const double* const*
             }
             if (launch_status() != GQ_OK) return GQ_ERR_CUDA;
         }
-        // 4. the recurrence over the rows of every weight of the group, 8 rows
-        // per block when their residuals fit in shared memory, else 4
-        const int rpb = gptq_rows_smem(nmax, 8) <= (size_t)kGptqSmemLimit ? 8 : 4;
-        GptqParams P;
-        std::memset(&P, 0, sizeof(P));
-        P.ndesc = gc;
-        int64_t blocks = 0;
-        for (int k = 0; k < gc; ++k) {
-            const int i = idx[g0 + k];
-            const gq_tensor& T = t[i];
-            GptqRowDesc& R = P.d[k];
-            R.w = T.w;
-            R.L = ws[g0 + k].L;
-            R.dead = ws[g0 + k].dead;
-            R.st = ws[g0 + k].st;
-            R.clip = ws[g0 + k].clip;
-            R.scale_f16 = T.scale_f16;
-            R.codes = T.codes;
-            R.packed = T.packed;
-            R.dq = T.dq;
-            R.status = d_status ? d_status + i : nullptr;
-            R.rows = T.rows;
-            R.n = T.cols;
-            R.ld = T.ld;
-            R.prb = packed_row_bytes(T.cols, T.qbits);
-            R.start = blocks;
-            R.dtype = T.dtype;
-            R.qbits = T.qbits;
-            blocks += (T.rows + rpb - 1) / rpb;
-        }
-        P.blocks = blocks;
-        if (P.blocks > INT32_MAX) return GQ_ERR_UNSUPPORTED;
-        const size_t smem = gptq_rows_smem(nmax, rpb);
+        // 4. the recurrence over the rows of every weight of the group: one
+        // launch per shared-memory class (blocks per SM that the residuals of
+        // a weight's columns allow), so that narrow weights are not given the
+        // shared memory, and the occupancy, of the widest
         int dev = 0;
         if (cudaGetDevice(&dev) != cudaSuccess) return GQ_ERR_CUDA;
-        const int ri = rpb == 8 ? 1 : 0;
-        if (dev >= 0 && dev < kMaxDevices && g_gptq_smem_set[ri][dev].load() < (int)smem) {
-            if (cuda_status(cudaFuncSetAttribute(ri ? gptq_rows_kernel<8> : gptq_rows_kernel<4>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != GQ_OK)
-                return GQ_ERR_CUDA;
-            g_gptq_smem_set[ri][dev].store((int)smem);
+        auto per_sm = [](int64_t cols) { return (int)std::min<int64_t>(8, 232448 / (int64_t)gptq_rows_smem(cols)); };
+        std::vector<int> classes;
+        for (int k = 0; k < gc; ++k) {
+            const int c = per_sm(t[idx[g0 + k]].cols);
+            if (std::find(classes.begin(), classes.end(), c) == classes.end()) classes.push_back(c);
         }
-        if (ri) gptq_rows_kernel<8><<<(unsigned)P.blocks, kGpThreads, smem, stream>>>(P);
-        else gptq_rows_kernel<4><<<(unsigned)P.blocks, kGpThreads, smem, stream>>>(P);
-        if (launch_status() != GQ_OK) return GQ_ERR_CUDA;
+        std::sort(classes.begin(), classes.end());            // the widest weights first
+        for (int cls : classes) {
+            GptqParams P;
+            std::memset(&P, 0, sizeof(P));
+            int64_t blocks = 0, ncls = 0;
+            int nd = 0;
+            for (int k = 0; k < gc; ++k) {
+                const int i = idx[g0 + k];
+                const gq_tensor& T = t[i];
+                if (per_sm(T.cols) != cls) continue;
+                GptqRowDesc& R = P.d[nd++];
+                R.w = T.w;
+                R.L = ws[g0 + k].L;
+                R.dead = ws[g0 + k].dead;
+                R.st = ws[g0 + k].st;
+                R.clip = ws[g0 + k].clip;
+                R.scale_f16 = T.scale_f16;
+                R.codes = T.codes;
+                R.packed = T.packed;
+                R.dq = T.dq;
+                R.status = d_status ? d_status + i : nullptr;
+                R.rows = T.rows;
+                R.n = T.cols;
+                R.ld = T.ld;
+                R.prb = packed_row_bytes(T.cols, T.qbits);
+                R.start = blocks;
+                R.dtype = T.dtype;
+                R.qbits = T.qbits;
+                blocks += (T.rows + kGpRows - 1) / kGpRows;
+                ncls = std::max(ncls, T.cols);
+            }
+            P.ndesc = nd;
+            P.blocks = blocks;
+            if (P.blocks > INT32_MAX) return GQ_ERR_UNSUPPORTED;
+            const size_t smem = gptq_rows_smem(ncls);
+            if (dev >= 0 && dev < kMaxDevices && g_gptq_smem_set[dev].load() < (int)smem) {
+                if (cuda_status(cudaFuncSetAttribute(gptq_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                     (int)smem)) != GQ_OK)
+                    return GQ_ERR_CUDA;
+                g_gptq_smem_set[dev].store((int)smem);
+            }
+            gptq_rows_kernel<<<(unsigned)P.blocks, kGpThreads, smem, stream>>>(P);
+            if (launch_status() != GQ_OK) return GQ_ERR_CUDA;
+        }
     }
     return GQ_OK;
 }

@@ -29,7 +29,7 @@
 //                        dead diagonals set to 1 first;
 //   gptq_chol_panel / gptq_chol_update  right-looking blocked Cholesky of
 //                        Hr in place (2 launches per 64-wide panel);
-//   gptq_rows_kernel     the recurrence, 4 or 8 rows per block, columns in
+//   gptq_rows_kernel     the recurrence, 4 rows per block, columns in
 //                        batches of 64: a dot-product pass over the earlier
 //                        columns' residuals, then the batch's columns in
 //                        order (one warp per row, one shuffle per column);
@@ -41,6 +41,7 @@
 namespace gq {
 
 constexpr int kGpBlock = 64;         // columns per batch of the recurrence / Cholesky panel width
+constexpr int kGpRows = 4;           // weight rows per block of the recurrence
 constexpr int kGpThreads = 256;
 constexpr int kGpHTile = 64;         // Hessian tile
 constexpr int kGpHChunk = 32;        // input rows per Hessian step
@@ -330,39 +331,33 @@ struct GptqParams {
     GptqRowDesc d[kGpMaxDesc];
 };
 
-// Shared memory of gptq_rows_kernel<R>: residuals of the block's rows over
-// all columns [R][n], the batch's scaled factor block [64][65], the partial
-// sums [R][64] and the batch's codes [R][64].
-__host__ __device__ inline size_t gptq_rows_smem(int64_t n, int rows_per_block) {
-    return (size_t)rows_per_block * (size_t)n * 8 + (size_t)kGpBlock * (kGpBlock + 1) * 8 +
-           (size_t)rows_per_block * kGpBlock * 8 + (size_t)rows_per_block * kGpBlock * 4;
+// Shared memory of gptq_rows_kernel: residuals of the block's rows over all
+// columns [kGpRows][n], the batch's scaled factor block [64][65], the
+// partial sums [kGpRows][64] and the batch's codes [kGpRows][64].
+__host__ __device__ inline size_t gptq_rows_smem(int64_t n) {
+    return (size_t)kGpRows * (size_t)n * 8 + (size_t)kGpBlock * (kGpBlock + 1) * 8 + (size_t)kGpRows * kGpBlock * 8 +
+           (size_t)kGpRows * kGpBlock * 4;
 }
 
-// R weight rows per block (4, or 8 when their residuals fit in shared
-// memory): in (a) each thread takes one column of the batch for R / 4 rows,
-// so that one load of the factor feeds R / 4 fused multiply-adds; in (b)
-// warp r owns row r.  Every sum keeps its order whatever R is.
-template <int R>
 __global__ void __launch_bounds__(kGpThreads) gptq_rows_kernel(const __grid_constant__ GptqParams P) {
-    static_assert(R == 4 || R == 8, "rows per block");
     extern __shared__ __align__(16) unsigned char gp_smem[];
     int di = 0;
     while (di + 1 < P.ndesc && (int64_t)blockIdx.x >= P.d[di + 1].start) ++di;
     const GptqRowDesc& D = P.d[di];
     const int64_t n = D.n;
-    const int64_t r0 = ((int64_t)blockIdx.x - D.start) * R;
-    const int nr = (int)min((int64_t)R, D.rows - r0);
-    double* res = reinterpret_cast<double*>(gp_smem);                     // [R][n]
-    double* Mb = res + (size_t)R * n;                                      // [64][65]
-    double* part = Mb + kGpBlock * (kGpBlock + 1);                         // [R][64]
-    int* qs = reinterpret_cast<int*>(part + R * kGpBlock);                 // [R][64]
+    const int64_t r0 = ((int64_t)blockIdx.x - D.start) * kGpRows;
+    const int nr = (int)min((int64_t)kGpRows, D.rows - r0);
+    double* res = reinterpret_cast<double*>(gp_smem);                     // [kGpRows][n]
+    double* Mb = res + (size_t)kGpRows * n;                                // [64][65]
+    double* part = Mb + kGpBlock * (kGpBlock + 1);                         // [kGpRows][64]
+    int* qs = reinterpret_cast<int*>(part + kGpRows * kGpBlock);           // [kGpRows][64]
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     const int qmax = D.qbits == 6 ? 31 : 127;
     const double* L = D.L;
 
     // row scales: the export's, from the clip of the original row
-    __shared__ double c_row[R], s_row[R];
-    if (t < R) {
+    __shared__ double c_row[kGpRows], s_row[kGpRows];
+    if (t < kGpRows) {
         c_row[t] = 0.0;
         s_row[t] = 0.0;
         if (t < nr) {
@@ -383,21 +378,14 @@ __global__ void __launch_bounds__(kGpThreads) gptq_rows_kernel(const __grid_cons
         // (a) the earlier columns' contribution: thread (r, jj) sums
         // res[r, i] * L[n-1-i, n-1-j] over i < j0, divided by V[j, j] below
         {
-            constexpr int RT = R / 4;                      // rows per thread
-            const int rq = t / kGpBlock, jj = t % kGpBlock;
-            double acc[RT];
-#pragma unroll
-            for (int k = 0; k < RT; ++k) acc[k] = 0.0;
-            if (rq < nr && jj < nb) {
+            const int r = t / kGpBlock, jj = t % kGpBlock;
+            double acc = 0.0;
+            if (r < nr && jj < nb) {
                 const int64_t colL = n - 1 - (j0 + jj);
-                for (int64_t i = 0; i < j0; ++i) {
-                    const double l = L[(n - 1 - i) * n + colL];
-#pragma unroll
-                    for (int k = 0; k < RT; ++k) acc[k] = __fma_rn(res[(size_t)(rq + 4 * k) * n + i], l, acc[k]);
-                }
+                const double* rr = res + (size_t)r * n;
+                for (int64_t i = 0; i < j0; ++i) acc = __fma_rn(rr[i], L[(n - 1 - i) * n + colL], acc);
             }
-#pragma unroll
-            for (int k = 0; k < RT; ++k) part[(rq + 4 * k) * kGpBlock + jj] = acc[k];
+            part[r * kGpBlock + jj] = acc;
         }
         // the batch's own factor block, scaled by its column's diagonal:
         // Mb[ii][jj] = V[j0+ii, j0+jj] / V[j0+jj, j0+jj] for ii < jj
@@ -459,7 +447,7 @@ __global__ void __launch_bounds__(kGpThreads) gptq_rows_kernel(const __grid_cons
         }
         __syncthreads();
         // (c) outputs of the batch: codes, w_hat, packed bytes
-        for (int e = t; e < R * kGpBlock; e += kGpThreads) {
+        for (int e = t; e < kGpRows * kGpBlock; e += kGpThreads) {
             const int r = e / kGpBlock, jj = e % kGpBlock;
             if (r >= nr || jj >= nb) continue;
             const int64_t grow = r0 + r, j = j0 + jj;
@@ -474,7 +462,7 @@ __global__ void __launch_bounds__(kGpThreads) gptq_rows_kernel(const __grid_cons
         }
         if (D.qbits == 6) {
             // 4 codes -> 3 bytes; batches are 64 wide, so groups never straddle
-            for (int e = t; e < R * (kGpBlock / 4); e += kGpThreads) {
+            for (int e = t; e < kGpRows * (kGpBlock / 4); e += kGpThreads) {
                 const int r = e / (kGpBlock / 4), g = e % (kGpBlock / 4);
                 if (r >= nr || 4 * g >= nb) continue;
                 uint32_t v = 0;
