@@ -1040,8 +1040,10 @@ gq_status gq_dequant(const uint8_t* d_packed, const uint16_t* d_scale_f16, int q
     const size_t vin = out_dtype == GQ_F32 ? 16 : 8;
     const int vec_out = aligned(d_out, vin) && ((cols * (int64_t)esz) % (int64_t)vin) == 0;
     const int words = aligned(d_packed, 4) && (qbits == 6 ? (cols % 16) == 0 : (cols % 4) == 0);
+    // one warp per row segment of 32 * kDqUnroll quads (the kernel's work items)
+    const int64_t segs = ((cols + 3) / 4 + 32 * kDqUnroll - 1) / (32 * kDqUnroll);
     const int64_t blocks = std::min<int64_t>((int64_t)sm_count() * 8,
-                                             (rows + kBlockWarps - 1) / kBlockWarps);
+                                             (rows * segs + kBlockWarps - 1) / kBlockWarps);
     dequant_kernel<<<(unsigned)blocks, kBlockThreads, 0, stream>>>(
         d_packed, d_scale_f16, qbits, gran == GQ_PER_TENSOR, rows, cols, prb, d_out, out_dtype,
         vec_out, words);

@@ -226,7 +226,7 @@ ste_kernel(const void* __restrict__ g_out, void* __restrict__ g_w, int dtype, in
 // 24-bit int6 groups are reassembled with two shuffles; otherwise bytes.
 // The code words of kDqUnroll steps are loaded before any of them is used,
 // so that a warp keeps that many loads in flight instead of one.
-constexpr int kDqUnroll = 4;
+constexpr int kDqUnroll = 8;
 
 __global__ void __launch_bounds__(kBlockThreads)
 dequant_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ sf16, int qbits,
@@ -240,12 +240,18 @@ dequant_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ 
     const int a = (3 * sub) >> 2;
     const int shift = 8 * ((3 * sub) & 3);
     const int nq = (int)((cols + 3) >> 2);
+    // work items: segments of one outer step (32 * kDqUnroll quads) of a row,
+    // so that long rows spread evenly over the warps
+    const int segs = (nq + 32 * kDqUnroll - 1) / (32 * kDqUnroll);
+    const int64_t items = rows * (int64_t)segs;
     const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += nwarps) {
+    for (int64_t it = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); it < items; it += nwarps) {
+        const int64_t r = it / segs;
+        const int jb0 = (int)(it - r * segs) * (32 * kDqUnroll);
         const uint16_t hb = sf16[per_tensor ? 0 : r];
         const float s = __half2float(*reinterpret_cast<const __half*>(&hb));
         const uint8_t* prow = packed + r * prb;
-        for (int jb0 = 0; jb0 < nq; jb0 += 32 * kDqUnroll) {
+        {
             // the code words (or bytes) of kDqUnroll steps, loaded first
             uint32_t raw[kDqUnroll];
 #pragma unroll
