@@ -93,15 +93,28 @@ ptsel_kernel(const __grid_constant__ SelParams P) {
                 }
             }
         };
-        int64_t i = tid;
-        for (; i + (int64_t)(kSelUnroll - 1) * kBlockThreads < nv; i += (int64_t)kSelUnroll * kBlockThreads) {
-            uint4 v[kSelUnroll];
+        // Whole rounds of kSelUnroll vectors per thread, double-buffered: the
+        // next round's loads are issued before this round is counted, so the
+        // load latency overlaps the counting instead of following it.
+        const int64_t step = (int64_t)kSelUnroll * kBlockThreads;
+        const int64_t rounds = nv / step;
+        uint4 va[kSelUnroll], vb[kSelUnroll];
+        auto load_round = [&](int64_t rd, uint4 (&v)[kSelUnroll]) {
 #pragma unroll
-            for (int u = 0; u < kSelUnroll; ++u) v[u] = src[i + (int64_t)u * kBlockThreads];
+            for (int u = 0; u < kSelUnroll; ++u) v[u] = src[rd * step + tid + (int64_t)u * kBlockThreads];
+        };
+        if (rounds > 0) load_round(0, va);
+        for (int64_t rd = 0; rd < rounds; rd += 2) {
+            if (rd + 1 < rounds) load_round(rd + 1, vb);
 #pragma unroll
-            for (int u = 0; u < kSelUnroll; ++u) count16(v[u]);
+            for (int u = 0; u < kSelUnroll; ++u) count16(va[u]);
+            if (rd + 1 < rounds) {
+                if (rd + 2 < rounds) load_round(rd + 2, va);
+#pragma unroll
+                for (int u = 0; u < kSelUnroll; ++u) count16(vb[u]);
+            }
         }
-        for (; i < nv; i += kBlockThreads) count16(src[i]);
+        for (int64_t i = rounds * step + tid; i < nv; i += kBlockThreads) count16(src[i]);
         const char* wb = reinterpret_cast<const char*>(D.w);
         for (int64_t e = e0 + nv * epv + tid; e < e1; e += kBlockThreads)
             count(D.dtype == kF32 ? reinterpret_cast<const float*>(wb)[e]
@@ -313,9 +326,11 @@ dequant_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ 
                 } else {
                     uint16_t* o = reinterpret_cast<uint16_t*>(out) + r * cols;
                     if (vec_out && full) {
-                        *reinterpret_cast<uint2*>(o + e0) =
-                            make_uint2((uint32_t)float_to_bf16_bits(d[0]) | ((uint32_t)float_to_bf16_bits(d[1]) << 16),
-                                       (uint32_t)float_to_bf16_bits(d[2]) | ((uint32_t)float_to_bf16_bits(d[3]) << 16));
+                        // two elements per conversion, each rounded to nearest even
+                        const __nv_bfloat162 lo = __floats2bfloat162_rn(d[0], d[1]);
+                        const __nv_bfloat162 hi = __floats2bfloat162_rn(d[2], d[3]);
+                        *reinterpret_cast<uint2*>(o + e0) = make_uint2(*reinterpret_cast<const uint32_t*>(&lo),
+                                                                       *reinterpret_cast<const uint32_t*>(&hi));
                     } else {
                         for (int i = 0; i < 4; ++i)
                             if (e0 + i < cols) o[e0 + i] = float_to_bf16_bits(d[i]);
