@@ -129,11 +129,17 @@ bool needs_workspace(const gq_tensor& t) {
     return t.qbits != 16 && t.gran == GQ_PER_TENSOR && t.rows > 0 && t.cols > 0;
 }
 
-size_t workspace_size(const gq_tensor* t, int n) {
+// A per-tensor group's workspace slot: the histogram and state (kWsSlot),
+// then, unless the caller has no room for it, kSelCand candidate keys.
+constexpr int32_t kSelCand = 4096;
+constexpr size_t kCandBytes = (size_t)kSelCand * 4;
+size_t slot_bytes(bool cand) { return kWsSlot + (cand ? kCandBytes : 0); }
+
+size_t workspace_size(const gq_tensor* t, int n, bool cand = true) {
     size_t slots = 0;
     for (int i = 0; i < n; ++i)
         if (needs_workspace(t[i])) ++slots;
-    return slots * kWsSlot;
+    return slots * slot_bytes(cand);
 }
 
 thread_local int g_last_cuda_error = 0;
@@ -349,7 +355,7 @@ gq_status run_passthrough(const std::vector<PassDesc>& pd, cudaStream_t stream) 
 // The shared driver of gq_row_clip_select, gq_fakequant_fwd and gq_export_pack.
 gq_status quantize_batch(const gq_tensor* t, int n, Op op, bool f16_mode, void* ws,
                          size_t ws_bytes, int32_t* d_status, cudaStream_t stream,
-                         const gq_avg* avg = nullptr) {
+                         const gq_avg* avg = nullptr, bool cand = true) {
     if (n < 0 || (n > 0 && !t)) return GQ_ERR_INVALID_ARG;
     if (op == Op::Average && n > 0 && !avg) return GQ_ERR_INVALID_ARG;
     for (int i = 0; i < n; ++i) {
@@ -357,7 +363,7 @@ gq_status quantize_batch(const gq_tensor* t, int n, Op op, bool f16_mode, void* 
         if (st != GQ_OK) return st;
         if (op == Op::Average && (st = check_avg(t[i], avg[i])) != GQ_OK) return st;
     }
-    const size_t need = workspace_size(t, n);
+    const size_t need = workspace_size(t, n, cand);
     if (need > 0) {
         if (!ws || ws_bytes < need) return GQ_ERR_WORKSPACE;
         if (!aligned(ws, 256)) return GQ_ERR_MISALIGNED;
@@ -432,12 +438,14 @@ gq_status quantize_batch(const gq_tensor* t, int n, Op op, bool f16_mode, void* 
         if (T.gran == GQ_PER_TENSOR) {
             flags |= kPerTensor;
             const int64_t numel = T.rows * T.cols;
-            uint8_t* base = static_cast<uint8_t*>(ws) + slot * kWsSlot;
+            uint8_t* base = static_cast<uint8_t*>(ws) + slot * slot_bytes(cand);
             ++slot;
             SelDesc S{};
             S.w = T.w;
             S.hist = reinterpret_cast<uint32_t*>(base);
             S.state = reinterpret_cast<uint32_t*>(base + kSelBins * sizeof(uint32_t));
+            S.cand = cand ? reinterpret_cast<uint32_t*>(base + kWsSlot) : nullptr;
+            S.cap = cand ? kSelCand : 0;
             S.status = status;
             S.rows = T.rows;
             S.cols = T.cols;
@@ -988,14 +996,14 @@ gq_status gq_export_pack(const gq_tensor* t, int n, void* d_ws, size_t ws_bytes,
 gq_status gq_export_pack_noalloc(const gq_tensor* t, int n, int32_t* d_status,
                                  cudaStream_t stream) {
     if (n < 0 || (n > 0 && !t)) return GQ_ERR_INVALID_ARG;
-    const size_t need = n > 0 ? workspace_size(t, n) : 0;
+    const size_t need = n > 0 ? workspace_size(t, n, false) : 0;   // no candidate buffers here
     if (need > kNoAllocBytes) return GQ_ERR_WORKSPACE;
     void* ws = nullptr;
     if (need > 0) {
         gq_status st = noalloc_scratch(&ws);
         if (st != GQ_OK) return st;
     }
-    return quantize_batch(t, n, Op::Export, true, ws, kNoAllocBytes, d_status, stream);
+    return quantize_batch(t, n, Op::Export, true, ws, kNoAllocBytes, d_status, stream, nullptr, false);
 }
 
 gq_status gq_test_arm_wait_expiry(int64_t tile, uint64_t wait_ns) {

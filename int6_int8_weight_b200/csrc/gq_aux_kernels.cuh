@@ -16,7 +16,11 @@ namespace gq {
 struct SelDesc {
     const void* w;
     uint32_t* hist;            // 2048 counters in the workspace
-    uint32_t* state;           // [0] prefix [1] remaining [2] ticket [3] key
+    uint32_t* state;           // [0] prefix [1] remaining [2] ticket [3] key [4] keys in the pass-0 bucket
+                               // [5] candidates collected [6] resolved after pass 1
+    uint32_t* cand;            // nullable: room for `cap` candidate keys (the pass-0 bucket's)
+    int32_t cap;
+    int32_t pad2;
     int32_t* status;
     int64_t rows, cols, ld;
     int64_t rows_per_item;
@@ -39,6 +43,10 @@ constexpr int kSelUnroll = 8;
 // PASS 0: digit = key bits 30..20; PASS 1: bits 19..9 among keys whose bits
 // 30..20 equal the chosen prefix; PASS 2: bits 8..0 among keys whose bits
 // 30..9 match.  One block per item (a block of rows of one tensor).
+// Candidates: when the pass-0 bucket holds at most `cap` keys, pass 1 also
+// collects them, and its last block finishes the select over them (the same
+// 9-bit histogram among the keys whose bits 30..9 match, so the same key);
+// pass 2 then returns at once for that tensor.
 template <int PASS>
 __global__ void __launch_bounds__(kBlockThreads)
 ptsel_kernel(const __grid_constant__ SelParams P) {
@@ -54,7 +62,9 @@ ptsel_kernel(const __grid_constant__ SelParams P) {
     for (int i = tid; i < kSelBins; i += kBlockThreads) h[i] = 0u;
     __syncthreads();
 
+    if (PASS == 2 && __ldcg(&D.state[6]) != 0u) return;     // resolved from the candidates
     const uint32_t prefix = PASS == 0 ? 0u : __ldcg(&D.state[0]);
+    const bool collect = PASS == 1 && D.cand != nullptr && __ldcg(&D.state[4]) <= (uint32_t)D.cap;
     const int64_t r0 = it * D.rows_per_item;
     const int64_t r1 = min(D.rows, r0 + D.rows_per_item);
     const int esz = D.dtype == kF32 ? 4 : 2;
@@ -65,7 +75,13 @@ ptsel_kernel(const __grid_constant__ SelParams P) {
             bad |= key >= 0x7F800000u;
             atomicAdd(&h[key >> 20], 1u);
         } else if (PASS == 1) {
-            if ((key >> 20) == prefix) atomicAdd(&h[(key >> 9) & 0x7FFu], 1u);
+            if ((key >> 20) == prefix) {
+                atomicAdd(&h[(key >> 9) & 0x7FFu], 1u);
+                if (collect) {
+                    const uint32_t idx = atomicAdd(&D.state[5], 1u);
+                    if (idx < (uint32_t)D.cap) D.cand[idx] = key;
+                }
+            }
         } else {
             if ((key >> 9) == prefix) atomicAdd(&h[key & 0x1FFu], 1u);
         }
@@ -174,6 +190,7 @@ ptsel_kernel(const __grid_constant__ SelParams P) {
                                         : ((prefix << 9) | (uint32_t)bin);
                 D.state[0] = np;
                 D.state[1] = (uint32_t)(rem - acc);
+                if (PASS == 0) D.state[4] = c;
                 if (PASS == 2) D.state[3] = np;
                 break;
             }
@@ -183,6 +200,50 @@ ptsel_kernel(const __grid_constant__ SelParams P) {
     __syncthreads();
     for (int i = tid; i < kSelBins; i += kBlockThreads) D.hist[i] = 0u;
     if (tid == 0) D.state[2] = 0u;
+    if (PASS == 1 && collect) {
+        // pass 2 over the collected keys: the 9-bit histogram of the keys
+        // whose bits 30..9 equal the prefix just chosen, then the pick
+        for (int i = tid; i < 512; i += kBlockThreads) h[i] = 0u;
+        __syncthreads();
+        const uint32_t p22 = __ldcg(&D.state[0]);
+        const int64_t rem2 = (int64_t)__ldcg(&D.state[1]);
+        const uint32_t ncand = min(__ldcg(&D.state[5]), (uint32_t)D.cap);
+        for (uint32_t i = tid; i < ncand; i += kBlockThreads) {
+            const uint32_t key = __ldcg(&D.cand[i]);
+            if ((key >> 9) == p22) atomicAdd(&h[key & 0x1FFu], 1u);
+        }
+        __syncthreads();
+        const int per2 = 512 / kBlockThreads;             // 2 bins per thread
+        uint32_t sum2 = 0;
+        for (int i = 0; i < per2; ++i) sum2 += h[511 - per2 * tid - i];
+        uint32_t incl2 = sum2;
+        for (int off = 1; off < 32; off <<= 1) {
+            uint32_t o = __shfl_up_sync(0xFFFFFFFFu, incl2, off);
+            if (lane >= off) incl2 += o;
+        }
+        __syncthreads();                                 // s_warp is reused
+        if (lane == 31) s_warp[warp] = incl2;
+        __syncthreads();
+        uint32_t wbase2 = 0;
+        for (int w = 0; w < warp; ++w) wbase2 += s_warp[w];
+        const int64_t excl2 = (int64_t)wbase2 + (int64_t)(incl2 - sum2);
+        if (excl2 < rem2 && rem2 <= excl2 + (int64_t)sum2) {
+            int64_t acc2 = excl2;
+            for (int i = 0; i < per2; ++i) {
+                const int bin = 511 - per2 * tid - i;
+                const uint32_t c = h[bin];
+                if (acc2 + c >= rem2) {
+                    const uint32_t key = (p22 << 9) | (uint32_t)bin;
+                    D.state[0] = key;
+                    D.state[1] = (uint32_t)(rem2 - acc2);
+                    D.state[3] = key;
+                    D.state[6] = 1u;
+                    break;
+                }
+                acc2 += c;
+            }
+        }
+    }
 }
 
 // ------------------------------------------------------------ elementwise --
