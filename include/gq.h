@@ -296,7 +296,10 @@ GQ_API gq_status gq_dequant(const uint8_t* d_packed, const uint16_t* d_scale_f16
  * weight [N, K] exported per row) and s[n] = (float)scale_f16[n].  W_hat is
  * the bf16 fake-quant weight the forward pass would multiply by; it is
  * rebuilt tile by tile in tensor memory (the MMA's A operand) and never
- * written out.
+ * written out.  Decode-sized batches (M <= 16) whose packed rows are a
+ * multiple of 16 bytes long run on a register-level kernel instead: each
+ * warp streams its weight rows by TMA and dequantizes them straight into
+ * mma.sync fragments (the same W_hat, the same bound).
  *   d_x      bf16 [M, ldx] activations, row-major, 16-byte aligned, ldx % 8 == 0
  *   d_packed [N, gq_packed_row_bytes(K, qbits)] bytes, 16-byte aligned (4-byte
  *            aligned when the row length is not a multiple of 16 bytes)
@@ -307,7 +310,8 @@ GQ_API gq_status gq_dequant(const uint8_t* d_packed, const uint16_t* d_scale_f16
  * All buffers are the caller's; the call allocates nothing, checks its
  * arguments on the host before launching, and runs asynchronously on
  * `stream` (one kernel launch, plus a memset of Y when the batch has few
- * tiles and their K ranges are split over blocks).
+ * tiles and their K ranges are split over blocks, and always on the
+ * decode-sized path).
  * Products are exact (bf16 x bf16) and accumulate in binary32 in the tensor
  * cores' order (two accumulators for small batches, partial sums of split K
  * ranges added into Y), so Y is not bitwise reproducible against a sequential
