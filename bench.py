@@ -963,6 +963,75 @@ def run_gemm(args):
                       "alg_gbs": round((wbytes + 2 * M * K + 4 * M * N) / us / 1e3, 1)}), flush=True)
 
 
+def run_batch(args):
+    """One model-shaped batched call alone (``--batch NAME``), for profiling
+    a single launch: ``gpt9`` (export of the 9-layer model), ``gpt12`` (mixed
+    per-row export of the 12-layer model), ``gpt12pt`` (per-tensor export of
+    its 72 block matrices) or ``unified11`` (bf16 training fake-quant of the
+    11-layer d528 model's 44 weights).  ``warmup`` then ``steps`` calls
+    through the C ABI, timed with CUDA events; one JSON line of its own."""
+    import torch
+    from int6_int8_weight_b200 import gq
+    device = torch.device("cuda")
+    if args.batch == "gpt9":
+        ws = synth.draw_gpt9()
+        items, export = [(s, ws[s.name], False) for s in synth.gpt9_specs()], True
+    elif args.batch == "gpt12":
+        ws = synth.draw_gpt12()
+        items, export = [(s, ws[s.name], s.per_tensor) for s in synth.gpt12_mixed_specs()], True
+    elif args.batch == "gpt12pt":
+        ws = synth.draw_gpt12()
+        items, export = [(s, ws[s.name], True) for s in synth.gpt12_mixed_specs() if s.qbits == 6], True
+    elif args.batch == "unified11":
+        ws = synth.draw_unified11()
+        items, export = [(s, ws[s.name].view(np.int16), False) for s in synth.unified11_train().specs], False
+    else:
+        raise SystemExit(f"unknown batch {args.batch!r}")
+    descs, keep = [], []
+    for spec, w, per_tensor in items:
+        W = torch.from_numpy(np.ascontiguousarray(w)).to(device)
+        if W.dtype == torch.int16:
+            W = W.view(torch.bfloat16)
+        if W.dim() == 1:
+            W = W.view(1, -1)
+        rows, cols = W.shape
+        keep.append(W)
+        if spec.qbits == 16:
+            o = torch.empty((rows, cols), dtype=torch.float16, device=device)
+            keep.append(o)
+            descs.append(gq.GQTensor(w=W.data_ptr(), dtype=gq._dtype_code(W), qbits=16, gran=0, reserved=0,
+                                     rows=rows, cols=cols, ld=cols, p=1.0, dq=0, codes=0, packed=o.data_ptr(),
+                                     scale_f16=0, scale_f32=0, clip=0))
+            continue
+        dq = torch.empty_like(W)
+        prb = gq.gq_packed_row_bytes(cols, spec.qbits)
+        pk = torch.empty((rows, prb), dtype=torch.uint8, device=device) if export else None
+        h = torch.empty(rows, dtype=torch.float16, device=device) if export else None
+        keep += [dq, pk, h]
+        descs.append(gq.GQTensor(w=W.data_ptr(), dtype=gq._dtype_code(W), qbits=spec.qbits,
+                                 gran=1 if per_tensor else 0, reserved=0, rows=rows, cols=cols, ld=cols,
+                                 p=spec.p, dq=dq.data_ptr(), codes=0, packed=pk.data_ptr() if export else 0,
+                                 scale_f16=h.data_ptr() if export else 0, scale_f32=0, clip=0))
+    arr = gq._arr(descs)
+    nb = gq.gq_workspace_size(descs)
+    wsb = torch.empty(max(nb, 256), dtype=torch.uint8, device=device)
+    if export:
+        fn = lambda: gq.LIB.gq_export_pack(arr, len(descs), wsb.data_ptr(), wsb.numel(), None, None)  # noqa: E731
+    else:
+        fn = lambda: gq.LIB.gq_fakequant_fwd(arr, len(descs), 0, wsb.data_ptr(), wsb.numel(), None, None)  # noqa: E731
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    print(json.dumps({"batch": args.batch, "tensors": len(descs),
+                      "us_per_call": round(a.elapsed_time(b) * 1e3 / max(args.steps, 1), 2)}), flush=True)
+
+
 def run_awq(args):
     """The AWQ column-scaled int6 export alone (``--awq ROWS,COLS``): a bf16
     synthetic weight, column scales from synthetic activation statistics,
@@ -1018,6 +1087,8 @@ def main(argv=None):
                     help="write profiles/rowquant_traffic.json from the ncu CSV of a --shrink run")
     ap.add_argument("--awq", default=None,
                     help="profile the AWQ column-scaled bf16 int6 export alone on ROWS,COLS (one JSON line of its own)")
+    ap.add_argument("--batch", default=None, choices=["gpt9", "gpt12", "gpt12pt", "unified11"],
+                    help="profile one model-shaped batched call alone (one JSON line of its own)")
     args = ap.parse_args(argv)
     if args.record_traffic:
         print(json.dumps(record_traffic(args.record_traffic, args.shrink), indent=1))
@@ -1027,6 +1098,9 @@ def main(argv=None):
         return
     if args.awq:
         run_awq(args)
+        return
+    if args.batch:
+        run_batch(args)
         return
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

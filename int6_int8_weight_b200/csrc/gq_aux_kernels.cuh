@@ -48,7 +48,7 @@ constexpr int kSelUnroll = 8;
 // 9-bit histogram among the keys whose bits 30..9 match, so the same key);
 // pass 2 then returns at once for that tensor.
 template <int PASS>
-__global__ void __launch_bounds__(kBlockThreads)
+__global__ void __launch_bounds__(kBlockThreads, 2)
 ptsel_kernel(const __grid_constant__ SelParams P) {
     __shared__ uint32_t h[kSelBins];
     __shared__ uint32_t s_warp[kBlockWarps];
@@ -109,28 +109,15 @@ ptsel_kernel(const __grid_constant__ SelParams P) {
                 }
             }
         };
-        // Whole rounds of kSelUnroll vectors per thread, double-buffered: the
-        // next round's loads are issued before this round is counted, so the
-        // load latency overlaps the counting instead of following it.
-        const int64_t step = (int64_t)kSelUnroll * kBlockThreads;
-        const int64_t rounds = nv / step;
-        uint4 va[kSelUnroll], vb[kSelUnroll];
-        auto load_round = [&](int64_t rd, uint4 (&v)[kSelUnroll]) {
+        int64_t i = tid;
+        for (; i + (int64_t)(kSelUnroll - 1) * kBlockThreads < nv; i += (int64_t)kSelUnroll * kBlockThreads) {
+            uint4 v[kSelUnroll];
 #pragma unroll
-            for (int u = 0; u < kSelUnroll; ++u) v[u] = src[rd * step + tid + (int64_t)u * kBlockThreads];
-        };
-        if (rounds > 0) load_round(0, va);
-        for (int64_t rd = 0; rd < rounds; rd += 2) {
-            if (rd + 1 < rounds) load_round(rd + 1, vb);
+            for (int u = 0; u < kSelUnroll; ++u) v[u] = src[i + (int64_t)u * kBlockThreads];
 #pragma unroll
-            for (int u = 0; u < kSelUnroll; ++u) count16(va[u]);
-            if (rd + 1 < rounds) {
-                if (rd + 2 < rounds) load_round(rd + 2, va);
-#pragma unroll
-                for (int u = 0; u < kSelUnroll; ++u) count16(vb[u]);
-            }
+            for (int u = 0; u < kSelUnroll; ++u) count16(v[u]);
         }
-        for (int64_t i = rounds * step + tid; i < nv; i += kBlockThreads) count16(src[i]);
+        for (; i < nv; i += kBlockThreads) count16(src[i]);
         const char* wb = reinterpret_cast<const char*>(D.w);
         for (int64_t e = e0 + nv * epv + tid; e < e1; e += kBlockThreads)
             count(D.dtype == kF32 ? reinterpret_cast<const float*>(wb)[e]
