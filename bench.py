@@ -198,7 +198,7 @@ def record_traffic(csv_path, shrink):
                     "each launch's bytes per row to the full row count"),
            "command": ("ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum "
                        f"--clock-control none -k regex:rowquant -s 36 -c 12 --csv --log-file "
-                       f"gpurun_out/step_traffic.csv python bench.py --shrink {shrink} --steps 1 "
+                       f"{csv_path} python bench.py --shrink {shrink} --steps 1 "
                        "--warmup 3 --skip-cpu --skip-rows --no-e2e")}
     with open(TRAFFIC_PATH, "w") as f:
         json.dump(out, f, indent=1)
