@@ -1025,40 +1025,86 @@ __device__ __forceinline__ void issue_tile(const TmaParams& P, int it, int& di, 
 // AWQ column scaling of one staged row, in place: element c becomes
 // RN_dtype(w * t[c]) -- one binary32 multiply, rounded to nearest even bf16
 // for a bf16 weight.  Thread `tl` of the row's `lpr` threads takes quads
-// tl, tl + lpr, ... (cols a multiple of 4).  The caller syncs the row's
-// threads before they read the row, after a proxy fence that orders these
-// generic stores before the next bulk copy into the stage.
+// tl, tl + lpr, ... (cols a multiple of 4), kScaleBatch at a time: the
+// batch's scale loads and shared-memory loads are all issued before its
+// first store, so their latencies overlap instead of adding up quad by quad.
+// The shared-memory accesses are volatile (kept in program order, loads of a
+// batch before its stores) but carry no memory clobber, so the scale loads
+// are free to move ahead of them.  Each thread touches only its own quads.
+// The caller syncs the row's threads before they read the row, after the
+// proxy fence here that orders these generic stores before the next bulk
+// copy into the stage.
+constexpr int kScaleBatch = 8;
+
+__device__ __forceinline__ void scale_quad_f32(uint32_t a, float4 c) {
+    float v0, v1, v2, v3;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v0), "=f"(v1), "=f"(v2), "=f"(v3) : "r"(a));
+    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(a), "f"(__fmul_rn(v0, c.x)),
+                 "f"(__fmul_rn(v1, c.y)), "f"(__fmul_rn(v2, c.z)), "f"(__fmul_rn(v3, c.w)));
+}
+
+__device__ __forceinline__ uint32_t scale_pair_bf16(uint32_t x, float c0, float c1) {
+    const __nv_bfloat162 r = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(x << 16), c0),
+                                                   __fmul_rn(__uint_as_float(x & 0xFFFF0000u), c1));
+    return *reinterpret_cast<const uint32_t*>(&r);
+}
+
 __device__ __forceinline__ void scale_row(uint32_t row, int cols, int dtype, const float* t, int tl, int lpr) {
     const int qpr = cols >> 2;
     const float4* t4 = reinterpret_cast<const float4*>(t);
-    // unrolled: several scale loads (L1 hits, but long-latency) in flight
-#pragma unroll 4
-    for (int j = tl; j < qpr; j += lpr) {
-        const float4 c = __ldg(t4 + j);
-        if (dtype == kF32) {
-            const uint32_t a = row + 16u * (uint32_t)j;
-            float v0, v1, v2, v3;
-            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                         : "=f"(v0), "=f"(v1), "=f"(v2), "=f"(v3)
-                         : "r"(a)
-                         : "memory");
-            asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(a), "f"(__fmul_rn(v0, c.x)),
-                         "f"(__fmul_rn(v1, c.y)), "f"(__fmul_rn(v2, c.z)), "f"(__fmul_rn(v3, c.w))
-                         : "memory");
-        } else {
+    int j = tl;
+    if (dtype == kF32) {
+        for (; j + (kScaleBatch - 1) * lpr < qpr; j += kScaleBatch * lpr) {
+            float4 c[kScaleBatch];
+            float v[kScaleBatch][4];
+#pragma unroll
+            for (int b = 0; b < kScaleBatch; ++b) c[b] = __ldg(t4 + j + b * lpr);
+#pragma unroll
+            for (int b = 0; b < kScaleBatch; ++b)
+                asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                             : "=f"(v[b][0]), "=f"(v[b][1]), "=f"(v[b][2]), "=f"(v[b][3])
+                             : "r"(row + 16u * (uint32_t)(j + b * lpr)));
+#pragma unroll
+            for (int b = 0; b < kScaleBatch; ++b)
+                asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(row + 16u * (uint32_t)(j + b * lpr)),
+                             "f"(__fmul_rn(v[b][0], c[b].x)), "f"(__fmul_rn(v[b][1], c[b].y)),
+                             "f"(__fmul_rn(v[b][2], c[b].z)), "f"(__fmul_rn(v[b][3], c[b].w)));
+        }
+        for (; j < qpr; j += lpr) scale_quad_f32(row + 16u * (uint32_t)j, __ldg(t4 + j));
+    } else {
+        for (; j + (kScaleBatch - 1) * lpr < qpr; j += kScaleBatch * lpr) {
+            float4 c[kScaleBatch];
+            uint32_t x[kScaleBatch], y[kScaleBatch];
+#pragma unroll
+            for (int b = 0; b < kScaleBatch; ++b) c[b] = __ldg(t4 + j + b * lpr);
+#pragma unroll
+            for (int b = 0; b < kScaleBatch; ++b)
+                asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];"
+                             : "=r"(x[b]), "=r"(y[b]) : "r"(row + 8u * (uint32_t)(j + b * lpr)));
+#pragma unroll
+            for (int b = 0; b < kScaleBatch; ++b)
+                asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(row + 8u * (uint32_t)(j + b * lpr)),
+                             "r"(scale_pair_bf16(x[b], c[b].x, c[b].y)), "r"(scale_pair_bf16(y[b], c[b].z, c[b].w)));
+        }
+        for (; j < qpr; j += lpr) {
+            const float4 c = __ldg(t4 + j);
             const uint32_t a = row + 8u * (uint32_t)j;
             uint32_t x, y;
-            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(x), "=r"(y) : "r"(a) : "memory");
-            const __nv_bfloat162 lo = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(x << 16), c.x),
-                                                            __fmul_rn(__uint_as_float(x & 0xFFFF0000u), c.y));
-            const __nv_bfloat162 hi = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(y << 16), c.z),
-                                                            __fmul_rn(__uint_as_float(y & 0xFFFF0000u), c.w));
-            asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(*reinterpret_cast<const uint32_t*>(&lo)),
-                         "r"(*reinterpret_cast<const uint32_t*>(&hi))
-                         : "memory");
+            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(x), "=r"(y) : "r"(a));
+            asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(scale_pair_bf16(x, c.x, c.y)),
+                         "r"(scale_pair_bf16(y, c.z, c.w)));
         }
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// The row's address after its in-place rescale and the sync that follows:
+// passed through a volatile asm placed after the sync, so that no read of the
+// rescaled row (plain asm loads, free to move) can be scheduled above it.
+__device__ __forceinline__ uint32_t launder_row(uint32_t row) {
+    uint32_t r;
+    asm volatile("mov.b32 %0, %1;" : "=r"(r) : "r"(row) : "memory");
+    return r;
 }
 
 // kColScale: the launch's descriptors all carry AWQ column scales (a
@@ -1158,22 +1204,25 @@ rowquant_tma_kernel(const __grid_constant__ TmaParams P) {
                 const int i = rd * slots + lslot;
                 const bool rv = i < nr;
                 const uint32_t row = stage + (uint32_t)(rv ? i : 0) * row_bytes;
+                uint32_t srow = row;
                 if constexpr (kColScale) {
                     // AWQ: the row becomes RN_dtype(w * t[c]) in place before its
                     // threads read it (the slots of a warp run in lockstep)
                     if (rv) scale_row(row, (int)D.cols, D.dtype, D.colscale, T.tl, lpr);
                     __syncwarp();
+                    srow = launder_row(row);
                 }
-                if (D.dtype == kF32) process_row_sub<kF32>(D, r0 + i, row, T, rv);
-                else process_row_sub<kBF16>(D, r0 + i, row, T, rv);
+                if (D.dtype == kF32) process_row_sub<kF32>(D, r0 + i, srow, T, rv);
+                else process_row_sub<kBF16>(D, r0 + i, srow, T, rv);
             }
         } else {
             for (int i = lslot; i < nr; i += slots, ++seq) {
-                const uint32_t row = stage + (uint32_t)i * row_bytes;
+                uint32_t row = stage + (uint32_t)i * row_bytes;
                 if constexpr (kColScale) {
                     scale_row(row, (int)D.cols, D.dtype, D.colscale, T.tl, lpr);
                     if (T.G > 1) T.team_sync();
                     else __syncwarp();
+                    row = launder_row(row);
                 }
                 uint32_t* bc = bcast + T.slot * kBcastWords;
                 uint32_t* hs = hist + T.slot * 256;
