@@ -443,7 +443,7 @@ def measure_rows(gq, device, peak):
     record("AWQ column-scaled export bf16 16384^2 int6 p=0.9999",
            timed(lambda: gq.LIB.gq_export_pack(arra, 1, None, 0, None, None)),
            4.75 * n + 2 * 16384 + 4 * 16384, 2 * n, 1,
-           note="reads w (2 B), writes w_hat (2 B) + packed (0.75 B); row kernel (reads the row twice)")
+           note="reads w (2 B), writes w_hat (2 B) + packed (0.75 B); pipelined row kernel, each staged row rescaled in place")
     del W, o, outd, Wb, dqb, avg, pk, h16, t_awq
 
     # the consuming GEMM with the int6 dequant in its weight load (tcgen05),
