@@ -1,6 +1,8 @@
 """Host-side bookkeeping of bench.py, without a GPU: the DRAM-traffic record
 written from the ncu CSV of one shrunken bandwidth-stress step, its scaling
-to full-size launches, and its withdrawal once the kernel sources change."""
+to full-size launches, and its withdrawal once the kernel sources change;
+the summary of the clock samples taken during the timed region (median SM
+clock under load, throttle reasons); the physical index of a rank's GPU."""
 import csv
 import json
 
@@ -110,3 +112,64 @@ def test_kernel_source_hash_covers_the_fused_kernel_sources():
     h = bench.kernel_source_hash()
     assert len(h) == 16 and h == bench.kernel_source_hash()
     assert "gq_rowquant_tma.cuh" in bench.FUSED_KERNEL_SOURCES
+
+
+class _Exited:
+    """Stands in for the nvidia-smi process of a ClockSampler."""
+
+    def terminate(self):
+        pass
+
+    def wait(self, timeout=None):
+        return 0
+
+    def kill(self):
+        pass
+
+
+def _sampler_over(tmp_path, lines):
+    s = bench.ClockSampler(0)
+    s.path = str(tmp_path / "clocks.csv")
+    with open(s.path, "w") as f:
+        f.write("\n".join(lines) + "\n")
+    s.proc = _Exited()
+    return s
+
+
+def test_clock_sampler_summary(tmp_path):
+    na, act = "Not Active", "Active"
+    lines = [
+        f"210, 1965, 95.1, 0x0000000000000001, {na}, {na}, {na}, {na}",      # idle before the region
+        f"1965, 1965, 812.0, 0x0000000000000000, {na}, {na}, {na}, {na}",
+        f"1950, 1965, 990.2, 0x0000000000000004, {na}, {na}, {na}, {act}",
+        f"1935, 1965, 1001.7, 0x0000000000000004, {na}, {na}, {na}, {act}",
+        "garbled line",
+    ]
+    out = _sampler_over(tmp_path, lines).stop()
+    assert out["samples"] == 4
+    assert out["sm_max_mhz"] == 1965.0
+    assert out["sm_mhz"] == 1950.0              # the idle 210 MHz sample is not "under load"
+    assert out["reasons"] == ["sw_power_cap"]
+    assert not set(out["reasons"]) & bench.REJECT
+
+
+def test_clock_sampler_reports_rejecting_reasons(tmp_path):
+    na, act = "Not Active", "Active"
+    lines = [f"1400, 1965, 1000.0, 0x0000000000000048, {act}, {na}, {act}, {na}"]
+    out = _sampler_over(tmp_path, lines).stop()
+    assert out["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
+    assert set(out["reasons"]) & bench.REJECT
+
+
+def test_clock_sampler_without_samples(tmp_path):
+    assert _sampler_over(tmp_path, ["[N/A]"]).stop() is None
+    assert bench.ClockSampler(0).stop() is None     # never started
+
+
+def test_physical_gpu_index(monkeypatch):
+    monkeypatch.setenv("CUDA_VISIBLE_DEVICES", "3, 5,7")
+    assert [bench.physical_gpu_index(r) for r in range(4)] == [3, 5, 7, 3]
+    monkeypatch.setenv("CUDA_VISIBLE_DEVICES", "GPU-1234abcd")
+    assert bench.physical_gpu_index(0) == 0
+    monkeypatch.delenv("CUDA_VISIBLE_DEVICES")
+    assert bench.physical_gpu_index(2) == 2
