@@ -2,7 +2,8 @@
 written from the ncu CSV of one shrunken bandwidth-stress step, its scaling
 to full-size launches, and its withdrawal once the kernel sources change;
 the summary of the clock samples taken during the timed region (median SM
-clock under load, throttle reasons); the physical index of a rank's GPU."""
+clock under load, throttle reasons); the physical index of a rank's GPU;
+the JSON line of the oracle reference arm, which runs on the host cores."""
 import csv
 import json
 
@@ -173,3 +174,29 @@ def test_physical_gpu_index(monkeypatch):
     assert bench.physical_gpu_index(0) == 0
     monkeypatch.delenv("CUDA_VISIBLE_DEVICES")
     assert bench.physical_gpu_index(2) == 2
+
+
+def test_reference_arm_json_line():
+    """`bench.py --impl reference` times the oracle on the host cores and
+    prints one JSON line in the bench contract; it needs no GPU."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "3"], capture_output=True, text=True, timeout=600, cwd=root)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["n_gpus"] == 1
+    assert line["steps"] == 1 and line["warmup"] == 3 and line["higher_is_better"] is True
+    assert line["value"] > 0 and line["unit"] == "GB/s" and line["ms_per_step"] > 0
+    assert line["config"]["workload"].startswith("bandwidth stress")
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"] and cb["value"] == line["value"]
+    e2e = line["e2e"]
+    assert e2e["value"] == line["value"] and e2e["unit"] == line["unit"]
+    assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+    # the minimum warm-up is enforced
+    bad = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--warmup", "2"],
+                         capture_output=True, text=True, timeout=120, cwd=root)
+    assert bad.returncode != 0 and "--warmup must be at least 3" in bad.stderr
